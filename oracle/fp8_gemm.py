@@ -1,0 +1,224 @@
+"""CPU oracle for the FP8 block-scaled GEMMs (test infrastructure only).
+
+This is the plain, slow, obviously correct definition of what the GPU path
+computes.  Only the test-suite, the package's smoke check and the benchmark's
+CPU-baseline leg may import it; the product path never does.  It shares no
+code with the CUDA library: it decodes every number format itself and uses
+NumPy's float64 matmul only as the inner product of one 128-wide K block.
+
+The operation (DeepGEMM pages, "细粒度缩放" / "两级累加结构" and the SF-format
+notes under "UE8M0 int32 packing"):
+
+    D[m, n] = bf16_rne( sum_kb  2^(ea[m,kb]-127) * 2^(eb[n//128,kb]-127)
+                               * sum_{k in block kb} e4m3(a[m,k]) * e4m3(b[n,k]) )
+
+where ea/eb are UE8M0 exponents unpacked from the int32 scale words.
+
+Exactness.  Every E4M3 value is a multiple of 2^-9, so every product is a
+multiple of 2^-18 and a 128-term block sum is bounded by 128*448^2 < 2^25:
+each block partial fits in 43 significant bits and is exact in float64 in any
+summation order, BLAS included.  Scaling by two powers of two is exact.  The
+only roundings are the float64 sum over K blocks (<= K/128 terms, relative
+error <= (K/128) * 2^-53) and the final round-to-nearest-even to BF16, done
+directly from float64 (no intermediate float32, so no double rounding).
+
+Parity pins: every function here is pinned in ``tests/test_oracle_pins.py``
+against closed forms, PyTorch's own FP8/BF16 conversions, brute force in
+exact rational arithmetic and integer arithmetic.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 128
+
+
+# ---------------------------------------------------------------------------
+# Number formats
+
+
+def e4m3_table() -> np.ndarray:
+    """Value of each of the 256 E4M3 ("E4M3FN") codes as float64.
+
+    Sign bit 7, exponent bits 6..3 (bias 7), mantissa bits 2..0.  Exponent 0
+    encodes subnormals m/8 * 2^-6; S.1111.111 is NaN; there is no infinity, so
+    the largest finite magnitude is 1.75 * 2^8 = 448.
+    """
+    codes = np.arange(256)
+    s = np.where(codes & 0x80, -1.0, 1.0)
+    e = (codes >> 3) & 0xF
+    m = codes & 0x7
+    sub = (m / 8.0) * 2.0 ** -6
+    nor = (1.0 + m / 8.0) * np.ldexp(1.0, e - 7)
+    v = s * np.where(e == 0, sub, nor)
+    v[(codes & 0x7F) == 0x7F] = np.nan
+    return v
+
+
+def ue8m0_value(e: np.ndarray) -> np.ndarray:
+    """2^(e-127) for UE8M0 exponent bytes (255 is NaN)."""
+    e = np.asarray(e).astype(np.int64)
+    v = np.ldexp(1.0, e - 127)
+    return np.where(e == 255, np.nan, v)
+
+
+def ue8m0_from_f32(sf: np.ndarray):
+    """UE8M0 byte of each fp32 scale; returns (bytes, bad_mask).
+
+    A valid scale is a positive finite power of two in the UE8M0 range:
+    normal fp32 powers of two give their biased exponent field, and the
+    subnormal 2^-127 gives 0.  Anything else is rejected (byte 0, bad=True).
+    """
+    bits = np.ascontiguousarray(sf, dtype=np.float32).view(np.uint32)
+    sign = bits >> 31
+    expf = (bits >> 23) & 0xFF
+    mant = bits & 0x7FFFFF
+    normal_ok = (sign == 0) & (expf >= 1) & (expf <= 254) & (mant == 0)
+    sub127 = (sign == 0) & (expf == 0) & (mant == 0x400000)  # 2^-127 = 2^22 * 2^-149
+    ok = normal_ok | sub127
+    byte = np.where(normal_ok, expf, 0).astype(np.uint8)
+    return byte, ~ok
+
+
+def packed_sf_shape(mn: int, kb: int):
+    """(words along K, words along MN) of one packed scale matrix."""
+    return (kb + 3) // 4, (mn + 3) // 4 * 4
+
+
+def pack_sf_ue8m0(sf: np.ndarray):
+    """Pack fp32 power-of-two scales [batch, MN, Kb] into UE8M0 int32 words.
+
+    Output int32 [batch, ceil(Kb/4), align4(MN)], MN contiguous ("transposed",
+    MN-major).  Byte j (bits 8j..8j+7, little-endian) of word [kp, mn] holds
+    the exponent of scale [mn, 4*kp + j].  Padding bytes (kb >= Kb, mn >= MN)
+    are 0.  Returns (words, number of rejected scales).
+    """
+    sf = np.asarray(sf, dtype=np.float32)
+    batch, mn, kb = sf.shape
+    byte, bad = ue8m0_from_f32(sf)
+    kp, mn4 = packed_sf_shape(mn, kb)
+    buf = np.zeros((batch, mn4, kp * 4), dtype=np.uint32)
+    buf[:, :mn, :kb] = byte
+    words = np.zeros((batch, kp, mn4), dtype=np.uint32)
+    for j in range(4):
+        words |= buf[:, :, j::4].transpose(0, 2, 1) << np.uint32(8 * j)
+    return words.view(np.int32), int(bad.sum())
+
+
+def unpack_sf_ue8m0(words: np.ndarray, mn: int, kb: int) -> np.ndarray:
+    """Inverse of :func:`pack_sf_ue8m0`: UE8M0 bytes [batch, MN, Kb]."""
+    w = np.asarray(words).view(np.uint32)
+    if w.ndim == 2:
+        w = w[None]
+    batch = w.shape[0]
+    out = np.zeros((batch, mn, kb), dtype=np.uint8)
+    for k in range(kb):
+        out[:, :, k] = ((w[:, k // 4, :mn] >> np.uint32(8 * (k % 4))) & 0xFF).astype(np.uint8)
+    return out
+
+
+def bf16_bits_from_f64(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to BF16 (round to nearest, ties to even); uint16 bits.
+
+    BF16 keeps 8 significant bits; its normal range starts at 2^-126 and its
+    subnormals are multiples of 2^-133.  For each x the quantum is
+    2^(floor(log2|x|) - 7) (or 2^-133 below the normal range); x is divided by
+    the quantum (exact: a power of two), rounded half-to-even to an integer
+    and scaled back, which is exact.  Results of magnitude >= 2^128 overflow
+    to infinity.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.float64)
+    fin = np.isfinite(x) & (x != 0)
+    _, ex = np.frexp(np.where(fin, x, 1.0))
+    lg = ex - 1  # floor(log2|x|)
+    qexp = np.where(lg < -126, -133, lg - 7)
+    q = np.rint(np.ldexp(np.where(fin, x, 0.0), -qexp))
+    r = np.ldexp(q, qexp)
+    r = np.where(np.abs(r) >= 2.0 ** 128, np.copysign(np.inf, x), r)
+    out[...] = np.where(fin, r, x)
+    f32 = out.astype(np.float32)  # exact: every r is a BF16 value
+    bits = (f32.view(np.uint32) >> 16).astype(np.uint16)
+    bits = np.where(np.isnan(x), np.uint16(0x7FC0), bits)
+    return bits.astype(np.uint16)
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+# ---------------------------------------------------------------------------
+# GEMMs
+
+
+def _decode(codes: np.ndarray) -> np.ndarray:
+    return e4m3_table()[np.asarray(codes, dtype=np.uint8)]
+
+
+def fp8_gemm_nt_f64(a, sfa_words, b, sfb_words, M, N, K, rows=None, cols=None) -> np.ndarray:
+    """Unrounded float64 D = A . B^T with per-128-K scale promotion.
+
+    a: uint8 [M,K] E4M3; b: uint8 [N,K] E4M3; sfa_words: int32 packed scales of
+    A (MN = M rows, one per 128 K); sfb_words: int32 packed scales of B (MN =
+    ceil(N/128) blocks).  ``rows``/``cols`` select a sub-block of D.
+    """
+    Kb = K // BLOCK
+    assert K % BLOCK == 0
+    ea = unpack_sf_ue8m0(sfa_words, M, Kb)[0]
+    eb = unpack_sf_ue8m0(sfb_words, (N + BLOCK - 1) // BLOCK, Kb)[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    cols = np.arange(N) if cols is None else np.asarray(cols)
+    A = _decode(a[rows])
+    B = _decode(b[cols])
+    acc = np.zeros((len(rows), len(cols)), dtype=np.float64)
+    for kb in range(Kb):
+        ks = slice(kb * BLOCK, (kb + 1) * BLOCK)
+        partial = A[:, ks] @ B[:, ks].T                  # exact (see module doc)
+        sa = ue8m0_value(ea[rows, kb])                    # [rows]
+        sb = ue8m0_value(eb[cols // BLOCK, kb])           # [cols]
+        acc += partial * sa[:, None] * sb[None, :]        # two exact power-of-two scalings
+    return acc
+
+
+def fp8_gemm_nt(a, sfa_words, b, sfb_words, M, N, K, rows=None, cols=None) -> np.ndarray:
+    """BF16 bits of D = A . B^T (dense NT layout, D row-major [M,N])."""
+    return bf16_bits_from_f64(fp8_gemm_nt_f64(a, sfa_words, b, sfb_words, M, N, K, rows, cols))
+
+
+def m_grouped_fp8_gemm_nt_contiguous(a, sfa_words, b, sfb_words, m_indices, d_bits, G, N, K):
+    """Contiguous M-grouped GEMM, written into ``d_bits`` (uint16 [M_total,N]) in place.
+
+    Row m with e = m_indices[m] >= 0 gets D[m] = A[m] . B[e]^T with A's row
+    scales and expert e's block scales; rows with e == -1 are not written.
+    Returns the number of rows with an out-of-range expert index (not written).
+    """
+    M_total = a.shape[0]
+    bad = 0
+    for e in range(G):
+        rows = np.nonzero(m_indices == e)[0]
+        if len(rows) == 0:
+            continue
+        d_bits[rows] = fp8_gemm_nt(a, sfa_words, b[e], sfb_words[e], M_total, N, K, rows=rows)
+    bad += int(((m_indices < -1) | (m_indices >= G)).sum())
+    return bad
+
+
+def m_grouped_fp8_gemm_nt_masked(a, sfa_words, b, sfb_words, masked_m, d_bits, G, M_max, N, K):
+    """Masked M-grouped GEMM, written into ``d_bits`` (uint16 [G,M_max,N]) in place.
+
+    For each expert g, rows m < masked_m[g] get D[g,m] = A[g,m] . B[g]^T; rows
+    m >= masked_m[g] are not written.  Counts outside [0, M_max] are clamped
+    into it; the number of such counts is returned.
+    """
+    bad = 0
+    for g in range(G):
+        mg = int(masked_m[g])
+        if mg < 0 or mg > M_max:
+            bad += 1
+            mg = min(max(mg, 0), M_max)
+        if mg == 0:
+            continue
+        d_bits[g, :mg] = fp8_gemm_nt(a[g], sfa_words[g], b[g], sfb_words[g], M_max, N, K,
+                                     rows=np.arange(mg))
+    return bad
