@@ -1,0 +1,472 @@
+#!/usr/bin/env python
+"""Benchmark of the FP8 block-scaled GEMM hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+pack the activation scales (fp32 power-of-two -> UE8M0 int32, the packing
+kernel) and run the GEMM (TMA ring -> block-scaled tcgen05 MMA -> epilogue)
+on them.  Weight scales are packed once, as a deployment would.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU)
+every rank runs its own independent problem (weak scaling, no collective on
+the data path); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP8 block-scaled GEMM TFLOPS (dense/grouped/masked) and % of B200 roofline"
+DEFAULT_WORKLOAD = "dense_4096x7168x2048"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+           0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+           0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end loop (0 = min(steps, 100))")
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------- helpers
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "moe_grouped_gemm_05_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """Per-launch DRAM bytes of the GEMM kernel from a committed ncu summary,
+    only if it was taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    ent = rec.get(workload)
+    if not ent or ent.get("kernel_hash") != kernel_source_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, torch_dev: int):
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._handle = None
+        try:
+            import pynvml
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(torch_dev).uuid)
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    self._handle = h
+                    break
+            if self._handle is None:
+                self._handle = pynvml.nvmlDeviceGetHandleByIndex(torch_dev)
+            self._nvml = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - clocks are best effort off the GPU machine
+            self._handle = None
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self._handle)
+                self.samples.append((time.time(), mhz, int(rs)))
+            except Exception:  # noqa: BLE001
+                pass
+            self._stop.wait(0.02)
+
+    def start(self):
+        if self._handle is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def stop(self):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        busy = [s for s in self.samples if not (s[2] & 0x1)] or self.samples
+        bits = 0
+        for s in busy:
+            bits |= s[2]
+        return {"sm_mhz": float(statistics.median(s[1] for s in busy)), "sm_max_mhz": self.max_mhz,
+                "reasons": [n for b, n in REASONS.items() if bits & b and b != 0x1], "samples": len(busy)}
+
+
+# ---------------------------------------------------------------- problems
+
+
+def algorithmic_bytes(p) -> float:
+    """Bytes the GEMM must move at least once: A rows read, B read, D written, scales."""
+    kb = p.K // 128
+    if p.kind == "dense":
+        return p.M * p.K + p.N * p.K + 2.0 * p.M * p.N + 4.0 * (p.M + (p.N + 127) // 128) * kb / 4
+    if p.kind == "contiguous":
+        v = p.valid_rows
+        return v * p.K + p.G * p.N * p.K + 2.0 * v * p.N
+    v = p.valid_rows
+    active = int((p.masked_m > 0).sum())
+    return v * p.K + active * p.N * p.K + 2.0 * v * p.N
+
+
+def bound_of(p) -> str:
+    flops = p.flops
+    return "tensor" if flops / algorithmic_bytes(p) > 560.0 else "hbm"
+
+
+def make_device_sets(p, dg, torch, dev):
+    """Device copies of one problem; enough copies that their total exceeds 2x L2."""
+    from moe_grouped_gemm_05_b200 import binding
+
+    a = torch.from_numpy(p.a).to(dev).view(torch.float8_e4m3fn)
+    b = torch.from_numpy(p.b).to(dev).view(torch.float8_e4m3fn)
+    sfa32 = torch.from_numpy(np.ascontiguousarray(p.sfa)).to(dev)
+    sfb32 = torch.from_numpy(np.ascontiguousarray(p.sfb)).to(dev)
+    if p.kind == "dense":
+        d_shape = (p.M, p.N)
+    elif p.kind == "contiguous":
+        d_shape = (p.M, p.N)
+    else:
+        d_shape = (p.G, p.M, p.N)
+    per_set = a.numel() + b.numel() + 2 * int(np.prod(d_shape))
+    nsets = max(1, -(-2 * L2_BYTES // per_set))
+    sets = []
+    for i in range(nsets):
+        s = {"a": a if i == 0 else a.clone(), "b": b if i == 0 else b.clone(),
+             "sfa32": sfa32 if i == 0 else sfa32.clone(),
+             "d": torch.empty(d_shape, dtype=torch.bfloat16, device=dev)}
+        s["sfb"] = binding.pack_sf_ue8m0(sfb32 if i == 0 else sfb32.clone())
+        s["sfa"] = binding.pack_sf_ue8m0(s["sfa32"])
+        if p.m_indices is not None:
+            s["m_indices"] = torch.from_numpy(p.m_indices).to(dev)
+        if p.masked_m is not None:
+            s["masked_m"] = torch.from_numpy(p.masked_m).to(dev)
+        sets.append(s)
+    return sets, per_set
+
+
+def gemm_call(p, dg, s):
+    if p.kind == "dense":
+        return dg.fp8_gemm_nt(s["a"], s["sfa"], s["b"], s["sfb"], s["d"])
+    if p.kind == "contiguous":
+        return dg.m_grouped_fp8_gemm_nt_contiguous(s["a"], s["sfa"], s["b"], s["sfb"], s["m_indices"], s["d"])
+    return dg.m_grouped_fp8_gemm_nt_masked(s["a"], s["sfa"], s["b"], s["sfb"], s["masked_m"], s["d"])
+
+
+def pack_call(dg, lib, s, torch):
+    """Packs the step's activation scales into s['sfa'] (the packing kernel, in place)."""
+    import ctypes
+
+    sf = s["sfa32"]
+    if sf.dim() == 2:
+        batch, mn, kb = 1, sf.shape[0], sf.shape[1]
+    else:
+        batch, mn, kb = sf.shape
+    code = lib.dg_pack_sf_ue8m0(ctypes.c_void_p(sf.data_ptr()), ctypes.c_void_p(s["sfa"].data_ptr()), batch, mn,
+                                kb, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    if code != 0:
+        raise RuntimeError(lib.dg_get_last_error().decode())
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+
+class OracleSample:
+    """The CPU oracle on a bounded row sample of a workload (all N, all K).
+
+    One run packs the sample rows' activation scales and computes their
+    output rows, i.e. the same two steps as one GPU step, on fewer rows."""
+
+    def __init__(self, p):
+        import oracle
+
+        self.oracle, self.p = oracle, p
+        if p.kind == "masked":
+            g = int(np.argmax(p.masked_m))
+            self.a, self.b, self.sfa32, sfb = p.a[g], p.b[g], p.sfa[g], p.sfb[g]
+            self.rows_total, self.desc = int(p.masked_m[g]), f"expert {g}"
+        elif p.kind == "contiguous":
+            self.a, self.b, self.sfa32, sfb = p.a, p.b[0], p.sfa, p.sfb[0]
+            self.rows_total, self.desc = int((p.m_indices == 0).sum()), "expert 0"
+        else:
+            self.a, self.b, self.sfa32, sfb = p.a, p.b, p.sfa, p.sfb
+            self.rows_total, self.desc = p.M, "the problem"
+        self.sfb = oracle.pack_sf_ue8m0(sfb[None])[0][0]  # weights: packed once
+        try:
+            from threadpoolctl import threadpool_info
+
+            self.cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        except Exception:  # noqa: BLE001
+            self.cores = os.cpu_count() or 1
+
+    def run(self, rows: int) -> float:
+        p, o = self.p, self.oracle
+        t0 = time.perf_counter()
+        sfa = o.pack_sf_ue8m0(self.sfa32[None, :rows])[0][0]
+        o.fp8_gemm_nt(self.a[:rows], sfa, self.b, self.sfb, rows, p.N, p.K)
+        return time.perf_counter() - t0
+
+    def calibrate(self, seconds: float) -> int:
+        r0 = max(1, min(self.rows_total, 16))
+        t0 = self.run(r0)
+        return int(max(1, min(self.rows_total, r0 * seconds / max(t0, 1e-6))))
+
+    def info(self, rows: int, t: float) -> dict:
+        p = self.p
+        return {"value": 2.0 * rows * p.N * p.K / t / 1e12, "unit": "TFLOPS", "cores": int(self.cores),
+                "kind": "oracle",
+                "sample": f"{p.name}: first {rows} valid rows of {self.desc} x all {p.N} columns x K={p.K}, "
+                          f"{t:.2f} s per run on host cores"}
+
+
+# ---------------------------------------------------------------- arms
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from moe_grouped_gemm_05_b200 import synth
+
+    p = synth.WORKLOADS[args.workload]()
+    total_steps = args.steps + args.warmup
+    per_step = max(0.05, min(2.0, 150.0 / max(total_steps, 1)))
+    smp = OracleSample(p)
+    rows = smp.calibrate(per_step)
+    times = []
+    for i in range(total_steps):
+        dt = smp.run(rows)
+        if i >= args.warmup:
+            times.append(dt)
+    step_s = statistics.mean(times) if times else smp.run(rows)
+    info = smp.info(rows, step_s)
+    value = info["value"]
+    line = {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": args.workload, "sample_rows": rows, "N": p.N, "K": p.K},
+            "impl": "reference", "cpu_baseline": info,
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from moe_grouped_gemm_05_b200 import binding as dg
+    from moe_grouped_gemm_05_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    lib = dg.load()
+    # rank r runs its own problem (seed offset): independent units, weak scaling
+    maker = synth.WORKLOADS[args.workload]
+    p = maker()
+    sets, per_set = make_device_sets(p, dg, torch, dev)
+    nsets = len(sets)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        s = sets[i % nsets]
+        pack_call(dg, lib, s, torch)
+        gemm_call(p, dg, s)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert dg.get_device_error() == 0, "device error word set during warm-up"
+
+    kernel_desc = dg.describe_config(p.kind, p.M, p.N, p.K, p.G)
+    ev_g0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_g1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local).start()
+    barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for i in range(args.steps):
+        s = sets[i % nsets]
+        pack_call(dg, lib, s, torch)
+        ev_g0[i].record(stream)
+        gemm_call(p, dg, s)
+        ev_g1[i].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    elapsed_ms = start.elapsed_time(end)
+    gemm_ms = [a.elapsed_time(b) for a, b in zip(ev_g0, ev_g1)]
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_ms = float(t.item())
+    err = dg.get_device_error()
+
+    # end to end through the public API: pinned host inputs in, result out, every step
+    e2e_steps = args.e2e_steps or min(args.steps, 100)
+    s0 = sets[0]
+    a_host = torch.from_numpy(p.a).pin_memory()
+    sfa_host = torch.from_numpy(np.ascontiguousarray(p.sfa)).pin_memory()
+    d_host = torch.empty(s0["d"].shape, dtype=torch.bfloat16).pin_memory()
+    h2d = a_host.numel() + sfa_host.numel() * 4
+    d2h = d_host.numel() * 2
+    for _ in range(2):
+        s0["a"].view(torch.uint8).copy_(a_host, non_blocking=True)
+        s0["sfa32"].copy_(sfa_host, non_blocking=True)
+        pack_call(dg, lib, s0, torch)
+        gemm_call(p, dg, s0)
+        d_host.copy_(s0["d"], non_blocking=True)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        s0["a"].view(torch.uint8).copy_(a_host, non_blocking=True)
+        s0["sfa32"].copy_(sfa_host, non_blocking=True)
+        pack_call(dg, lib, s0, torch)
+        gemm_call(p, dg, s0)
+        d_host.copy_(s0["d"], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = float(e2e_ms.item())
+
+    flops = p.flops
+    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    gemm_avg_ms = statistics.mean(gemm_ms)
+    bound = bound_of(p)
+    long_region = elapsed_ms > 500.0
+    if bound == "tensor":
+        bf16 = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+        peak = 2.0 * bf16  # FP8 dense = 2 x BF16 dense (nominal ratio)
+        achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        peak_note = (f"{'sustained' if long_region else 'burst'} bf16 x2 ({peak_src})")
+    else:
+        peak = peaks.get("hbm_gbs")
+        achieved = algorithmic_bytes(p) / (gemm_avg_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        peak_note = f"copy bandwidth ({peak_src})"
+    traffic = recorded_traffic(args.workload)
+    clocks = sampler.summary()
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
+        "config": {"workload": args.workload, "kind": p.kind, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
+                   "valid_rows": p.valid_rows, "kernel_config": kernel_desc,
+                   "step": "pack activation scales (fp32 -> UE8M0 int32) + GEMM",
+                   "l2": f"inputs rotate over {nsets} device copies ({nsets * per_set / 1e6:.0f} MB > 2x L2)"},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                     "frac": achieved / peak if peak else None, "traffic": traffic, "peak_source": peak_note,
+                     "kernel": "fp8_gemm_kernel", "kernel_ms_avg": gemm_avg_ms,
+                     "kernel_ms_min": min(gemm_ms)},
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": e2e_steps},
+        "gpu_launches": 2 * args.steps,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "device_error": err,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        smp = OracleSample(p)
+        rows = smp.calibrate(args.cpu_seconds)
+        line["cpu_baseline"] = smp.info(rows, smp.run(rows))
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

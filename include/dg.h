@@ -1,0 +1,151 @@
+/*
+ * dg.h — C ABI of the B200 (sm_100a) FP8 block-scaled GEMM library (libdg.so).
+ *
+ * Operation (DeepGEMM pages: "DeepGEMM 简介" and "4 DeepGEMM 架构分析 — 两级累加结构"
+ * on the juejin.cn Open-Source-Week article; "Per-block scaling 通过 CUDA-core
+ * promotion" and "UE8M0 int32 packing" on the nightvoyager.top GitHub report):
+ *
+ *   D[m,n] = bf16_rne( sum_kb sa[m,kb] * sb[n/128,kb]
+ *                             * sum_{k in 128-wide block kb} A[m,k] * B[n,k] )
+ *
+ * A, B are FP8 E4M3; sa is one power-of-two scale per row of A and 128-wide K
+ * block (1x128), sb one per 128x128 block of B; both are UE8M0 exponents
+ * packed four per int32.  D is BF16, overwritten (no C input).
+ *
+ * Conventions shared by every entry point
+ *  - Every data pointer is DEVICE memory owned by the caller, 16-byte aligned.
+ *    The library allocates nothing per call; it keeps only a per-device
+ *    error word.  `stream` is a cudaStream_t (NULL = legacy default stream);
+ *    calls are asynchronous and stream-ordered.
+ *  - Layouts are row-major and dense.  "NT": A is [M,K] and B is [N,K], both
+ *    K-contiguous; D is [M,N], N-contiguous.
+ *  - Packed scales ("TMA-aligned, transposed" layout of the ssnai.com DeepGEMM
+ *    analysis, FP8 pitfalls block): a matrix of scales with MN rows and Kb = K/128
+ *    blocks is stored as int32 words [ceil(Kb/4)][align4(MN)], MN contiguous;
+ *    byte j (bits 8j..8j+7) of word [kp][mn] is the UE8M0 exponent e of block
+ *    4*kp+j, meaning 2^(e-127).  Padding bytes are 0.  For A, MN = rows of A;
+ *    for B, MN = ceil(N/128).
+ *  - Requirements: K % 128 == 0 and K > 0; N % 16 == 0 and N > 0; M >= 0.
+ *  - Return value: DG_OK or a negative dg_status.  Argument errors are found on
+ *    the host before anything is launched (the C counterpart of DeepGEMM's
+ *    host asserts); dg_get_last_error() then describes the problem.
+ *    Data-dependent errors (expert index out of range, masked_m outside
+ *    [0, M_max], a scale that is not a power of two) are found on the device:
+ *    the kernel skips or clamps the offending item, sets a bit in the device
+ *    error word and returns normally.  Read it with dg_get_device_error().
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  DG_OK = 0,
+  DG_ERR_NULL = -1,        /* a required pointer is NULL                     */
+  DG_ERR_SHAPE = -2,       /* a size violates the requirements above         */
+  DG_ERR_ALIGN = -3,       /* a pointer is not 16-byte aligned               */
+  DG_ERR_UNSUPPORTED = -4, /* no GPU / not sm_100 / configuration not built  */
+  DG_ERR_CUDA = -5,        /* a CUDA runtime or driver call failed           */
+  DG_ERR_DEVICE_DATA = -6, /* reported by dg_get_device_error                */
+  DG_ERR_TIMEOUT = -7      /* reported by dg_get_device_error                */
+} dg_status;
+
+/* Bits of the device error word. */
+#define DG_DEVERR_BAD_SCALE     0x1  /* pack: a scale is not a power of two in UE8M0 range */
+#define DG_DEVERR_BAD_EXPERT    0x2  /* contiguous: m_indices value < -1 or >= num_groups  */
+#define DG_DEVERR_BAD_MASKED_M  0x4  /* masked: masked_m[g] < 0 or > M_max (clamped)       */
+#define DG_DEVERR_MIXED_TILE    0x8  /* contiguous: a 128-row tile holds two experts       */
+#define DG_DEVERR_TIMEOUT       0x10 /* a pipeline wait exceeded its time limit; CTA quit   */
+
+/*
+ * Dense FP8 GEMM, NT layout (juejin.cn article §5 "常规稠密 GEMM"; the
+ * nightvoyager.top report's "fp8_gemm_nt(a, b, d, c=None, ...)" signature).
+ *   a   : E4M3 [M][K]                 sfa : packed scales, MN = M
+ *   b   : E4M3 [N][K]                 sfb : packed scales, MN = ceil(N/128)
+ *   d   : BF16 [M][N], written in full (M == 0 is a no-op).
+ */
+int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream);
+
+/*
+ * M-grouped GEMM, contiguous layout (juejin.cn article §4 "分组 GEMM（连续布局）":
+ * the experts' tokens are concatenated along M, each expert segment aligned
+ * to the M block; N and K are shared by all experts).
+ *   a         : E4M3 [M_total][K]     sfa : packed scales, MN = M_total
+ *   b         : E4M3 [G][N][K]        sfb : G packed matrices, MN = ceil(N/128)
+ *   d         : BF16 [M_total][N]
+ *   m_indices : int32 [M_total], expert of each row, -1 for padding rows.
+ * M_total must be a multiple of 128 (dg_get_mk_alignment_for_contiguous_layout)
+ * and every aligned 128-row tile must hold rows of one expert (plus -1 rows).
+ * Rows with index -1 are not written.  A tile whose first row is -1 is
+ * skipped entirely.  Out-of-range indices set DG_DEVERR_BAD_EXPERT and their
+ * rows are not written; rows of a second expert inside a tile set
+ * DG_DEVERR_MIXED_TILE and are not written.
+ */
+int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                        const int32_t* sfb, void* d, const int32_t* m_indices,
+                                        int M_total, int N, int K, int num_groups, void* stream);
+
+/*
+ * M-grouped GEMM, masked layout (juejin.cn article §4 "分组 GEMM（掩码分组）":
+ * fixed per-expert capacity plus a device-side valid count, so the call can be
+ * captured in a CUDA graph while token counts change).
+ *   a        : E4M3 [G][M_max][K]     sfa : G packed matrices, MN = M_max
+ *   b        : E4M3 [G][N][K]         sfb : G packed matrices, MN = ceil(N/128)
+ *   d        : BF16 [G][M_max][N]
+ *   masked_m : int32 [G] on the device, valid rows of each expert; read by the
+ *              kernel, never by the host.  Rows m >= masked_m[g] of expert g
+ *              are not written.  Values outside [0, M_max] are clamped and set
+ *              DG_DEVERR_BAD_MASKED_M.
+ */
+int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
+                                    const int32_t* sfb, void* d, const int32_t* masked_m,
+                                    int num_groups, int M_max, int N, int K, void* stream);
+
+/*
+ * Packs fp32 power-of-two scales into the UE8M0 int32 layout above
+ * (nightvoyager.top report, "SF 双 path 缓存设计": float32 scales go through a
+ * transform kernel once, e.g. for weights, and the packed words are reused).
+ *   sf     : fp32 [batch][mn][kb]          (device)
+ *   packed : int32 [batch][ceil(kb/4)][align4(mn)]   (device, fully written)
+ * A valid scale is a positive normal fp32 power of two, or 2^-127 (byte 0).
+ * Anything else writes byte 0 and sets DG_DEVERR_BAD_SCALE.
+ */
+int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb, void* stream);
+
+/* M alignment of expert segments in the contiguous layout (128). */
+int dg_get_mk_alignment_for_contiguous_layout(void);
+
+/* Number of int32 words of one packed scale matrix: ceil(kb/4) * align4(mn). */
+int64_t dg_packed_sf_words(int mn, int kb);
+
+/* Synchronises `stream`, returns the current device's error word in *err
+ * (0 = none, else DG_DEVERR_* bits) and clears it. */
+int dg_get_device_error(void* stream, int* err);
+
+/* Persistent-grid size (the ssnai.com analysis' set_num_sms knob).
+ * n <= 0 restores "all SMs".  Returns the previous setting. */
+int dg_set_num_sms(int n);
+int dg_get_num_sms(void);
+
+/* Forces the tile configuration of the next calls on this host thread:
+ * block_n (a built N tile width) and stages (0 = largest that fits).
+ * block_n == 0 restores the heuristic.  Returns DG_OK or DG_ERR_UNSUPPORTED. */
+int dg_set_config(int block_n, int stages);
+
+/* Describes the configuration the heuristic picks for a problem, as
+ * "BMxBNxSTAGES/grid" in buf (kind: 0 dense, 1 contiguous, 2 masked). */
+int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf, int buflen);
+
+/* Text of the last host-side error on this thread ("" if none). */
+const char* dg_get_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */

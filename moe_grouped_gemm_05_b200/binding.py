@@ -1,0 +1,191 @@
+"""Thin ctypes binding of libdg.so (argument marshalling only).
+
+Every step of the GEMM runs in the library's CUDA kernels; this module checks
+tensor dtypes/shapes, passes raw device pointers and the current CUDA stream,
+and turns negative status codes into exceptions.  Tensors come from PyTorch
+(device memory and streams only).  If the library is missing the first call
+raises: there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libdg.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "dg.h")
+
+DG_DEVERR_BAD_SCALE = 0x1
+DG_DEVERR_BAD_EXPERT = 0x2
+DG_DEVERR_BAD_MASKED_M = 0x4
+DG_DEVERR_MIXED_TILE = 0x8
+DG_DEVERR_TIMEOUT = 0x10
+
+_lib = None
+
+
+class DGError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"dg status {code}: {msg}")
+        self.code = code
+
+
+def load() -> ctypes.CDLL:
+    """Loads libdg.so once (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m moe_grouped_gemm_05_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i32p, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
+    lib.dg_fp8_gemm_nt.argtypes = [vp, i32p, vp, i32p, vp, i, i, i, vp]
+    lib.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
+    lib.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
+    lib.dg_pack_sf_ue8m0.argtypes = [vp, i32p, i, i, i, vp]
+    lib.dg_packed_sf_words.argtypes = [i, i]
+    lib.dg_packed_sf_words.restype = ctypes.c_int64
+    lib.dg_get_mk_alignment_for_contiguous_layout.argtypes = []
+    lib.dg_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
+    lib.dg_set_num_sms.argtypes = [i]
+    lib.dg_get_num_sms.argtypes = []
+    lib.dg_set_config.argtypes = [i, i]
+    lib.dg_describe_config.argtypes = [i, i, i, i, i, ctypes.c_char_p, i]
+    lib.dg_get_last_error.restype = ctypes.c_char_p
+    for name in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous", "dg_m_grouped_fp8_gemm_nt_masked",
+                 "dg_pack_sf_ue8m0", "dg_get_device_error", "dg_set_config", "dg_describe_config"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/dg.h."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dg_\w+)\s*\(", text)))
+
+
+def _check(code: int):
+    if code != 0:
+        raise DGError(code, load().dg_get_last_error().decode())
+
+
+def _stream() -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _ptr(t: torch.Tensor) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _fp8(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise TypeError(f"{name} must be float8_e4m3fn (or its uint8 bytes), got {t.dtype}")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return t
+
+
+def _i32(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+        raise TypeError(f"{name} must be a contiguous int32 CUDA tensor")
+    return t
+
+
+def packed_sf_words(mn: int, kb: int) -> tuple[int, int]:
+    """(rows, cols) of a packed scale matrix: (ceil(kb/4), align4(mn))."""
+    return (kb + 3) // 4, (mn + 3) // 4 * 4
+
+
+def pack_sf_ue8m0(sf: torch.Tensor) -> torch.Tensor:
+    """fp32 power-of-two scales [batch?, mn, kb] -> int32 [batch?, ceil(kb/4), align4(mn)]."""
+    if sf.dtype != torch.float32 or not sf.is_cuda or not sf.is_contiguous():
+        raise TypeError("sf must be a contiguous float32 CUDA tensor")
+    squeeze = sf.dim() == 2
+    s3 = sf.unsqueeze(0) if squeeze else sf
+    if s3.dim() != 3:
+        raise ValueError("sf must be [mn, kb] or [batch, mn, kb]")
+    batch, mn, kb = s3.shape
+    kp, mn4 = packed_sf_words(mn, kb)
+    out = torch.empty((batch, kp, mn4), dtype=torch.int32, device=sf.device)
+    _check(load().dg_pack_sf_ue8m0(_ptr(s3), _ptr(out), batch, mn, kb, _stream()))
+    return out[0] if squeeze else out
+
+
+def fp8_gemm_nt(a, sfa, b, sfb, d=None) -> torch.Tensor:
+    """D[M,N] (bf16) = A[M,K] . B[N,K]^T with packed 1x128 / 128x128 UE8M0 scales."""
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb")
+    M, K = a.shape
+    N, Kb_ = b.shape
+    if Kb_ != K:
+        raise ValueError("a and b disagree on K")
+    if tuple(sfa.shape) != packed_sf_words(M, K // 128) or tuple(sfb.shape) != packed_sf_words(-(-N // 128), K // 128):
+        raise ValueError("packed scale shapes do not match [ceil(Kb/4), align4(MN)]")
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
+        raise ValueError("d must be a contiguous bf16 [M, N] tensor")
+    _check(load().dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices, d=None) -> torch.Tensor:
+    """Contiguous-layout grouped GEMM: D[m] = A[m] . B[m_indices[m]]^T; -1 rows untouched."""
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb"), _i32(m_indices, "m_indices")
+    M, K = a.shape
+    G, N, Kb_ = b.shape
+    if Kb_ != K or m_indices.shape != (M,):
+        raise ValueError("shape mismatch")
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
+        raise ValueError("d must be a contiguous bf16 [M_total, N] tensor")
+    _check(load().dg_m_grouped_fp8_gemm_nt_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d),
+                                                       _ptr(m_indices), M, N, K, G, _stream()))
+    return d
+
+
+def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m, d=None) -> torch.Tensor:
+    """Masked-layout grouped GEMM: rows m < masked_m[g] of expert g; other rows untouched."""
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb"), _i32(masked_m, "masked_m")
+    G, M_max, K = a.shape
+    Gb, N, Kb_ = b.shape
+    if Gb != G or Kb_ != K or masked_m.shape != (G,):
+        raise ValueError("shape mismatch")
+    if d is None:
+        d = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=a.device)
+    elif d.dtype != torch.bfloat16 or tuple(d.shape) != (G, M_max, N) or not d.is_contiguous():
+        raise ValueError("d must be a contiguous bf16 [G, M_max, N] tensor")
+    _check(load().dg_m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d),
+                                                   _ptr(masked_m), G, M_max, N, K, _stream()))
+    return d
+
+
+def get_device_error() -> int:
+    """Synchronises the current stream, returns and clears the device error word."""
+    v = ctypes.c_int(0)
+    _check(load().dg_get_device_error(_stream(), ctypes.byref(v)))
+    return v.value
+
+
+def set_num_sms(n: int) -> int:
+    return load().dg_set_num_sms(n)
+
+
+def set_config(block_n: int, stages: int = 0) -> None:
+    _check(load().dg_set_config(block_n, stages))
+
+
+def describe_config(kind: str, M: int, N: int, K: int, num_groups: int = 1) -> str:
+    buf = ctypes.create_string_buffer(64)
+    k = {"dense": 0, "contiguous": 1, "masked": 2}[kind]
+    _check(load().dg_describe_config(k, M, N, K, num_groups, buf, 64))
+    return buf.value.decode()
+
+
+def get_mk_alignment_for_contiguous_layout() -> int:
+    return load().dg_get_mk_alignment_for_contiguous_layout()

@@ -1,0 +1,473 @@
+// Host side of libdg.so: argument validation, tensor maps, the tile
+// heuristic, kernel launches, the UE8M0 scale-packing kernel and the
+// device error word.  See include/dg.h for the contract of each entry point.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/dg.h"
+#include "fp8_gemm_kernel.cuh"
+
+namespace dg {
+
+// ------------------------------------------------------------------ errors
+
+static thread_local char t_last_error[512] = "";
+
+static int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(t_last_error, sizeof(t_last_error), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+#define DG_CUDA_TRY(expr)                                                               \
+  do {                                                                                  \
+    cudaError_t e_ = (expr);                                                            \
+    if (e_ != cudaSuccess)                                                              \
+      return fail(DG_ERR_CUDA, "%s failed: %s", #expr, cudaGetErrorString(e_));         \
+  } while (0)
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// ------------------------------------------------------------------ device info
+
+static int g_num_sms_override = 0;
+static thread_local int t_force_bn = 0;
+
+struct DeviceInfo {
+  int sms = 0;
+  int major = 0, minor = 0;
+  int max_smem = 0;
+};
+
+static int device_info(DeviceInfo* out) {
+  int dev = 0;
+  DG_CUDA_TRY(cudaGetDevice(&dev));
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  static bool have[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return fail(DG_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  if (!have[dev]) {
+    DeviceInfo d;
+    DG_CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    DG_CUDA_TRY(cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev));
+    DG_CUDA_TRY(cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev));
+    DG_CUDA_TRY(cudaDeviceGetAttribute(&d.max_smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    cache[dev] = d;
+    have[dev] = true;
+  }
+  *out = cache[dev];
+  if (out->major != 10 || out->minor != 0)
+    return fail(DG_ERR_UNSUPPORTED, "sm_%d%d device: this library is built for sm_100a only",
+                out->major, out->minor);
+  return DG_OK;
+}
+
+// ------------------------------------------------------------------ tensor maps
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 3-D tiled map: dims {d0 (contiguous), d1, d2}, byte strides of d1 and d2, box {b0, b1, 1}.
+static int make_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, uint64_t d0,
+                    uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0,
+                    uint32_t b1, CUtensorMapSwizzle swz, const char* what) {
+  auto fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {stride1, stride2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(DG_ERR_CUDA, "tensor map for %s rejected (CUresult %d; dims %llu x %llu x %llu)", what,
+                static_cast<int>(r), (unsigned long long)d0, (unsigned long long)d1,
+                (unsigned long long)d2);
+  return DG_OK;
+}
+
+// ------------------------------------------------------------------ configurations
+
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
+
+struct Config {
+  int bn = 0;
+  int stages = 0;
+  int smem = 0;
+  KernelFn fn = nullptr;
+};
+
+template <int BN, int STAGES, int MODE>
+static Config make_config() {
+  Config c;
+  c.bn = BN;
+  c.stages = STAGES;
+  c.smem = Layout<BN, STAGES>::kSmemBytes;
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE>);
+  return c;
+}
+
+template <int MODE>
+static const Config* config_table(int* count) {
+  static const Config table[] = {
+      make_config<128, 6, MODE>(), make_config<224, 4, MODE>(), make_config<256, 4, MODE>(),
+  };
+  *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
+  return table;
+}
+
+template <int MODE>
+static const Config* find_config(int bn) {
+  int n = 0;
+  const Config* t = config_table<MODE>(&n);
+  for (int i = 0; i < n; ++i)
+    if (t[i].bn == bn) return &t[i];
+  return nullptr;
+}
+
+// Heuristic: estimated time = waves x per-tile cost, where a 128 x BN tile
+// costs BN (tensor-core time) plus a fixed per-tile overhead for the
+// pipeline fill and epilogue; ragged N tiles waste their missing columns.
+template <int MODE>
+static const Config* choose_config(long long m_tiles_est, int N, int sms) {
+  if (t_force_bn) return find_config<MODE>(t_force_bn);
+  int n = 0;
+  const Config* t = config_table<MODE>(&n);
+  const Config* best = nullptr;
+  double best_cost = 1e300;
+  for (int i = 0; i < n; ++i) {
+    const int bn = t[i].bn;
+    const long long n_tiles = (N + bn - 1) / bn;
+    const long long tiles = m_tiles_est * n_tiles;
+    const long long waves = (tiles + sms - 1) / sms;
+    const double cost = static_cast<double>(waves) * (bn + 48.0);
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = &t[i];
+    }
+  }
+  return best;
+}
+
+static int raster_group(int num_m_blocks) { return std::min(num_m_blocks, 16); }
+
+template <int MODE>
+static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const GemmArgs& args,
+                  cudaStream_t stream) {
+  static std::mutex mu;
+  static bool attr_done[16] = {};
+  int idx = 0;
+  {
+    int n = 0;
+    const Config* t = config_table<MODE>(&n);
+    idx = static_cast<int>(cfg - t);
+  }
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_done[idx]) {
+      DG_CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(cfg->fn),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, cfg->smem));
+      attr_done[idx] = true;
+    }
+  }
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(grid);
+  lc.blockDim = dim3(kThreads);
+  lc.dynamicSmemBytes = cfg->smem;
+  lc.stream = stream;
+  DG_CUDA_TRY(cudaLaunchKernelEx(&lc, cfg->fn, maps[0], maps[1], maps[2], maps[3], maps[4], args));
+  return DG_OK;
+}
+
+// Builds the five tensor maps of one call.
+//   A   : [GA][rowsA][K] bytes           box 128 x 128, 128-byte swizzle
+//   B   : [GB][N][K] bytes               box 128 x BN,  128-byte swizzle
+//   SFA : [GA][Kp][align4(rowsA)] int32  box 128 words
+//   SFB : [GB][Kp][align4(Nb)] int32     box 8 words
+//   D   : [GD][rowsD][N] bf16            box 32 x 32,   64-byte swizzle
+static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const int32_t* sfa,
+                      const void* b, const int32_t* sfb, void* d, int rowsA, int GA, int N, int K,
+                      int GB, int rowsD, int GD) {
+  const uint64_t Kp = (K / 128 + 3) / 4;
+  const uint64_t mn4a = (static_cast<uint64_t>(rowsA) + 3) / 4 * 4;
+  const uint64_t nb4 = (static_cast<uint64_t>((N + 127) / 128) + 3) / 4 * 4;
+  int r;
+  if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, rowsA, GA, K,
+                    static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A")))
+    return r;
+  if ((r = make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K, N, GB, K,
+                    static_cast<uint64_t>(N) * K, 128, cfg->bn, CU_TENSOR_MAP_SWIZZLE_128B, "B")))
+    return r;
+  if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_INT32, sfa, mn4a, Kp, GA, mn4a * 4,
+                    Kp * mn4a * 4, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE, "SFA")))
+    return r;
+  if ((r = make_map(&maps[3], CU_TENSOR_MAP_DATA_TYPE_INT32, sfb, nb4, Kp, GB, nb4 * 4,
+                    Kp * nb4 * 4, 8, 1, CU_TENSOR_MAP_SWIZZLE_NONE, "SFB")))
+    return r;
+  if ((r = make_map(&maps[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, rowsD, GD,
+                    static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(rowsD) * N * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B, "D")))
+    return r;
+  return DG_OK;
+}
+
+static int check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
+                        void* d, int N, int K) {
+  if (!a || !sfa || !b || !sfb || !d) return fail(DG_ERR_NULL, "a, sfa, b, sfb and d must be non-NULL");
+  if (!aligned16(a) || !aligned16(b) || !aligned16(d) || !aligned16(sfa) || !aligned16(sfb))
+    return fail(DG_ERR_ALIGN, "a, sfa, b, sfb and d must be 16-byte aligned");
+  if (K <= 0 || K % 128 != 0) return fail(DG_ERR_SHAPE, "K=%d must be a positive multiple of 128", K);
+  if (N <= 0 || N % 16 != 0) return fail(DG_ERR_SHAPE, "N=%d must be a positive multiple of 16", N);
+  return DG_OK;
+}
+
+static int grid_size(int sms, long long tiles) {
+  int g = g_num_sms_override > 0 ? std::min(g_num_sms_override, sms) : sms;
+  if (tiles < g) g = static_cast<int>(std::max<long long>(tiles, 1));
+  return g;
+}
+
+// ------------------------------------------------------------------ pack kernel
+
+__global__ void pack_sf_ue8m0_kernel(const float* __restrict__ sf, uint32_t* __restrict__ out,
+                                     int batch, int mn, int kb, int kp, int mn4) {
+  const long long total = static_cast<long long>(batch) * kp * mn4;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int m = static_cast<int>(i % mn4);
+    const long long rest = i / mn4;
+    const int p = static_cast<int>(rest % kp);
+    const int bt = static_cast<int>(rest / kp);
+    uint32_t word = 0;
+    bool bad = false;
+    if (m < mn) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int k = 4 * p + j;
+        if (k >= kb) break;
+        const uint32_t bits = __float_as_uint(sf[(static_cast<long long>(bt) * mn + m) * kb + k]);
+        const uint32_t expf = (bits >> 23) & 0xFFu;
+        const uint32_t mant = bits & 0x7FFFFFu;
+        uint32_t byte = 0;
+        if ((bits >> 31) == 0 && expf >= 1 && expf <= 254 && mant == 0) {
+          byte = expf;
+        } else if (bits == 0x00400000u) {  // 2^-127, the fp32 subnormal of UE8M0 byte 0
+          byte = 0;
+        } else {
+          bad = true;
+        }
+        word |= byte << (8 * j);
+      }
+    }
+    out[i] = word;
+    if (bad) atomicOr(&g_dg_error, DG_DEVERR_BAD_SCALE);
+  }
+}
+
+}  // namespace dg
+
+using namespace dg;
+
+// ==================================================================== C ABI
+
+extern "C" {
+
+int dg_get_mk_alignment_for_contiguous_layout(void) { return kBM; }
+
+int64_t dg_packed_sf_words(int mn, int kb) {
+  if (mn < 0 || kb < 0) return -1;
+  return static_cast<int64_t>((kb + 3) / 4) * ((static_cast<int64_t>(mn) + 3) / 4 * 4);
+}
+
+const char* dg_get_last_error(void) { return t_last_error; }
+
+int dg_set_num_sms(int n) {
+  const int prev = g_num_sms_override;
+  g_num_sms_override = n > 0 ? n : 0;
+  return prev;
+}
+
+int dg_get_num_sms(void) {
+  DeviceInfo di;
+  if (device_info(&di) != DG_OK) return g_num_sms_override;
+  return g_num_sms_override > 0 ? std::min(g_num_sms_override, di.sms) : di.sms;
+}
+
+int dg_set_config(int block_n, int stages) {
+  if (block_n == 0) {
+    t_force_bn = 0;
+    return DG_OK;
+  }
+  if (!find_config<MODE_DENSE>(block_n)) return fail(DG_ERR_UNSUPPORTED, "block_n=%d is not built", block_n);
+  if (stages != 0 && stages != find_config<MODE_DENSE>(block_n)->stages)
+    return fail(DG_ERR_UNSUPPORTED, "block_n=%d is built with %d stages only", block_n,
+                find_config<MODE_DENSE>(block_n)->stages);
+  t_force_bn = block_n;
+  return DG_OK;
+}
+
+int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf, int buflen) {
+  (void)K;
+  if (!buf || buflen <= 0) return fail(DG_ERR_NULL, "buf must be non-NULL");
+  DeviceInfo di;
+  int sms = 148;
+  if (device_info(&di) == DG_OK) sms = di.sms;
+  if (g_num_sms_override > 0) sms = std::min(sms, g_num_sms_override);
+  if (N <= 0) return fail(DG_ERR_SHAPE, "N must be positive");
+  long long mt;
+  if (kind == 2) mt = static_cast<long long>(num_groups) * ((M + kBM - 1) / kBM);
+  else mt = (M + kBM - 1) / kBM;
+  const Config* c = kind == 1 ? choose_config<MODE_CONTIG>(mt, N, sms)
+                    : kind == 2 ? choose_config<MODE_MASKED>(mt, N, sms)
+                                : choose_config<MODE_DENSE>(mt, N, sms);
+  if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
+  const long long tiles = mt * ((N + c->bn - 1) / c->bn);
+  snprintf(buf, buflen, "%dx%dx%d/%d", kBM, c->bn, c->stages, grid_size(sms, tiles));
+  return DG_OK;
+}
+
+int dg_get_device_error(void* stream, int* err) {
+  if (!err) return fail(DG_ERR_NULL, "err must be non-NULL");
+  DG_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int v = 0;
+  DG_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_dg_error, sizeof(int)));
+  const int zero = 0;
+  DG_CUDA_TRY(cudaMemcpyToSymbol(g_dg_error, &zero, sizeof(int)));
+  *err = v;
+  return DG_OK;
+}
+
+int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb, void* stream) {
+  if (!sf || !packed) return fail(DG_ERR_NULL, "sf and packed must be non-NULL");
+  if (batch < 0 || mn < 0 || kb < 0) return fail(DG_ERR_SHAPE, "negative size");
+  if (!aligned16(packed)) return fail(DG_ERR_ALIGN, "packed must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(sf) & 3) != 0) return fail(DG_ERR_ALIGN, "sf must be 4-byte aligned");
+  const int kp = (kb + 3) / 4;
+  const int mn4 = (mn + 3) / 4 * 4;
+  const long long total = static_cast<long long>(batch) * kp * mn4;
+  if (total == 0) return DG_OK;
+  DeviceInfo di;
+  int r = device_info(&di);
+  if (r) return r;
+  const int threads = 256;
+  const long long blocks = std::min<long long>((total + threads - 1) / threads, 8LL * di.sms);
+  pack_sf_ue8m0_kernel<<<static_cast<int>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
+      sf, reinterpret_cast<uint32_t*>(packed), batch, mn, kb, kp, mn4);
+  DG_CUDA_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream) {
+  int r = check_common(a, sfa, b, sfb, d, N, K);
+  if (r) return r;
+  if (M < 0) return fail(DG_ERR_SHAPE, "M=%d must be >= 0", M);
+  if (M == 0) return DG_OK;
+  DeviceInfo di;
+  if ((r = device_info(&di))) return r;
+  const int mt = (M + kBM - 1) / kBM;
+  const Config* cfg = choose_config<MODE_DENSE>(mt, N, di.sms);
+  if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
+  CUtensorMap maps[5];
+  if ((r = build_maps(maps, cfg, a, sfa, b, sfb, d, M, 1, N, K, 1, M, 1))) return r;
+  GemmArgs args = {};
+  args.rows = M;
+  args.N = N;
+  args.K = K;
+  args.G = 1;
+  args.num_m_blocks = mt;
+  args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
+  args.raster_m = raster_group(mt);
+  args.d = static_cast<__nv_bfloat16*>(d);
+  const long long tiles = static_cast<long long>(mt) * args.num_n_blocks;
+  return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles), maps, args, static_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                        const int32_t* sfb, void* d, const int32_t* m_indices,
+                                        int M_total, int N, int K, int num_groups, void* stream) {
+  int r = check_common(a, sfa, b, sfb, d, N, K);
+  if (r) return r;
+  if (!m_indices) return fail(DG_ERR_NULL, "m_indices must be non-NULL");
+  if (num_groups <= 0) return fail(DG_ERR_SHAPE, "num_groups=%d must be positive", num_groups);
+  if (M_total < 0 || M_total % kBM != 0)
+    return fail(DG_ERR_SHAPE, "M_total=%d must be a non-negative multiple of %d", M_total, kBM);
+  if (M_total == 0) return DG_OK;
+  DeviceInfo di;
+  if ((r = device_info(&di))) return r;
+  const int mt = M_total / kBM;
+  const Config* cfg = choose_config<MODE_CONTIG>(mt, N, di.sms);
+  if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
+  CUtensorMap maps[5];
+  if ((r = build_maps(maps, cfg, a, sfa, b, sfb, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
+  GemmArgs args = {};
+  args.rows = M_total;
+  args.N = N;
+  args.K = K;
+  args.G = num_groups;
+  args.num_m_blocks = mt;
+  args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
+  args.raster_m = raster_group(mt);
+  args.m_indices = m_indices;
+  args.d = static_cast<__nv_bfloat16*>(d);
+  const long long tiles = static_cast<long long>(mt) * args.num_n_blocks;
+  return launch<MODE_CONTIG>(cfg, grid_size(di.sms, tiles), maps, args, static_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
+                                    const int32_t* sfb, void* d, const int32_t* masked_m,
+                                    int num_groups, int M_max, int N, int K, void* stream) {
+  int r = check_common(a, sfa, b, sfb, d, N, K);
+  if (r) return r;
+  if (!masked_m) return fail(DG_ERR_NULL, "masked_m must be non-NULL");
+  if (num_groups <= 0 || num_groups > kMaxMaskedGroups)
+    return fail(DG_ERR_SHAPE, "num_groups=%d must be in [1, %d]", num_groups, kMaxMaskedGroups);
+  if (M_max < 0) return fail(DG_ERR_SHAPE, "M_max=%d must be >= 0", M_max);
+  if (M_max == 0) return DG_OK;
+  DeviceInfo di;
+  if ((r = device_info(&di))) return r;
+  const int mt_per = (M_max + kBM - 1) / kBM;
+  // the device decides the real tile count; the heuristic assumes half-full experts
+  const long long mt_est = std::max<long long>(1, static_cast<long long>(num_groups) * mt_per / 2);
+  const Config* cfg = choose_config<MODE_MASKED>(mt_est, N, di.sms);
+  if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
+  CUtensorMap maps[5];
+  if ((r = build_maps(maps, cfg, a, sfa, b, sfb, d, M_max, num_groups, N, K, num_groups, M_max,
+                      num_groups)))
+    return r;
+  GemmArgs args = {};
+  args.rows = M_max;
+  args.N = N;
+  args.K = K;
+  args.G = num_groups;
+  args.num_m_blocks = mt_per;
+  args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
+  args.raster_m = 1;
+  args.masked_m = masked_m;
+  args.d = static_cast<__nv_bfloat16*>(d);
+  const long long max_tiles = static_cast<long long>(num_groups) * mt_per * args.num_n_blocks;
+  return launch<MODE_MASKED>(cfg, grid_size(di.sms, max_tiles), maps, args, static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,81 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects
+bad arguments on the host before touching the GPU (runs without a GPU)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from moe_grouped_gemm_05_b200 import binding, build
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return binding.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = binding.header_functions()
+    assert "dg_fp8_gemm_nt" in names and "dg_pack_sf_ue8m0" in names
+    out = subprocess.run(["nm", "-D", "--defined-only", binding.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(lib, n)
+
+
+def test_pure_host_queries(lib):
+    assert lib.dg_get_mk_alignment_for_contiguous_layout() == 128
+    assert lib.dg_packed_sf_words(4096, 16) == 4 * 4096
+    assert lib.dg_packed_sf_words(56, 16) == 4 * 56
+    assert lib.dg_packed_sf_words(13, 7) == 2 * 16
+    assert lib.dg_packed_sf_words(-1, 3) == -1
+
+
+P = ctypes.c_void_p
+GOOD = P(0x10000)
+
+
+def _dense(lib, a=GOOD, sfa=GOOD, b=GOOD, sfb=GOOD, d=GOOD, M=128, N=256, K=256):
+    return lib.dg_fp8_gemm_nt(a, sfa, b, sfb, d, M, N, K, None)
+
+
+def test_dense_argument_errors(lib):
+    assert _dense(lib, a=P(0)) == -1
+    assert b"non-NULL" in lib.dg_get_last_error()
+    assert _dense(lib, b=P(0x10008)) == -3
+    assert _dense(lib, K=100) == -2
+    assert b"K=100" in lib.dg_get_last_error()
+    assert _dense(lib, K=0) == -2
+    assert _dense(lib, N=200) == -2
+    assert _dense(lib, M=-5) == -2
+    assert _dense(lib, M=0) == 0  # empty problem: nothing to do, nothing launched
+
+
+def test_grouped_argument_errors(lib):
+    f = lib.dg_m_grouped_fp8_gemm_nt_contiguous
+    assert f(GOOD, GOOD, GOOD, GOOD, GOOD, P(0), 256, 256, 256, 4, None) == -1
+    assert f(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 200, 256, 256, 4, None) == -2
+    assert f(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 256, 256, 256, 0, None) == -2
+    assert f(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 0, 256, 256, 4, None) == 0
+    g = lib.dg_m_grouped_fp8_gemm_nt_masked
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, P(0), 4, 256, 256, 256, None) == -1
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 0, 256, 256, 256, None) == -2
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 100000, 256, 256, 256, None) == -2
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 4, 256, 256, 384 + 1, None) == -2
+    assert g(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 4, 0, 256, 256, None) == 0
+
+
+def test_pack_argument_errors(lib):
+    f = lib.dg_pack_sf_ue8m0
+    assert f(P(0), GOOD, 1, 4, 4, None) == -1
+    assert f(GOOD, P(0x10004), 1, 4, 4, None) == -3
+    assert f(GOOD, GOOD, -1, 4, 4, None) == -2
+    assert f(GOOD, GOOD, 0, 4, 4, None) == 0
+
+
+def test_config_override(lib):
+    assert lib.dg_set_config(96, 0) == -4
+    assert lib.dg_set_config(128, 0) == 0
+    assert lib.dg_set_config(0, 0) == 0
