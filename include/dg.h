@@ -133,12 +133,14 @@ int dg_set_num_sms(int n);
 int dg_get_num_sms(void);
 
 /* Forces the tile configuration of the next calls on this host thread:
- * block_n (a built N tile width) and stages (0 = largest that fits).
- * block_n == 0 restores the heuristic.  Returns DG_OK or DG_ERR_UNSUPPORTED. */
-int dg_set_config(int block_n, int stages);
+ * block_n (a built N tile width) and ctas (1: 128-row tiles on one SM;
+ * 2: 256-row tiles on a pair of SMs; 0: whichever is built, 1 first).
+ * block_n == 0 restores the heuristic.  The contiguous layout only has
+ * 1-CTA tiles.  Returns DG_OK or DG_ERR_UNSUPPORTED. */
+int dg_set_config(int block_n, int ctas);
 
 /* Describes the configuration the heuristic picks for a problem, as
- * "BMxBNxSTAGES/grid" in buf (kind: 0 dense, 1 contiguous, 2 masked). */
+ * "BMxBNxSTAGES[(2cta)]/grid" in buf (kind: 0 dense, 1 contiguous, 2 masked). */
 int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf, int buflen);
 
 /* Text of the last host-side error on this thread ("" if none). */

@@ -176,8 +176,9 @@ def set_num_sms(n: int) -> int:
     return load().dg_set_num_sms(n)
 
 
-def set_config(block_n: int, stages: int = 0) -> None:
-    _check(load().dg_set_config(block_n, stages))
+def set_config(block_n: int, ctas: int = 0) -> None:
+    """Forces the N tile width and 1- or 2-CTA tiles (block_n=0: heuristic)."""
+    _check(load().dg_set_config(block_n, ctas))
 
 
 def describe_config(kind: str, M: int, N: int, K: int, num_groups: int = 1) -> str:

@@ -11,7 +11,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/dg.h"
+#include "dg.h"
 #include "fp8_gemm_kernel.cuh"
 
 namespace dg {
@@ -109,62 +109,88 @@ static int make_map(CUtensorMap* map, CUtensorMapDataType type, const void* base
 
 // ------------------------------------------------------------------ configurations
 
-using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
+using KernelFn = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, GemmArgs);
 
 struct Config {
   int bn = 0;
   int stages = 0;
+  int ctas = 1;
   int smem = 0;
+  int num_acc = 1;
   KernelFn fn = nullptr;
 };
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int CTAS>
 static Config make_config() {
   Config c;
   c.bn = BN;
   c.stages = STAGES;
-  c.smem = Layout<BN, STAGES>::kSmemBytes;
-  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE>);
+  c.ctas = CTAS;
+  c.smem = Layout<BN, STAGES, CTAS>::kSmemBytes;
+  c.num_acc = Layout<BN, STAGES, CTAS>::kNumAcc;
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS>);
   return c;
 }
 
+// Built configurations.  A 2-CTA tile spans 256 rows, which the contiguous
+// layout (128-row expert alignment) cannot guarantee to be one expert, so the
+// contiguous mode uses single-CTA tiles only.
 template <int MODE>
 static const Config* config_table(int* count) {
-  static const Config table[] = {
-      make_config<128, 6, MODE>(), make_config<224, 4, MODE>(), make_config<256, 4, MODE>(),
-  };
-  *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
-  return table;
+  if constexpr (MODE == MODE_CONTIG) {
+    static const Config table[] = {
+        make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
+    };
+    *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
+    return table;
+  } else {
+    static const Config table[] = {
+        make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
+        make_config<128, 6, MODE, 2>(), make_config<224, 6, MODE, 2>(), make_config<256, 6, MODE, 2>(),
+    };
+    *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
+    return table;
+  }
 }
 
 template <int MODE>
-static const Config* find_config(int bn) {
+static const Config* find_config(int bn, int ctas) {
   int n = 0;
   const Config* t = config_table<MODE>(&n);
   for (int i = 0; i < n; ++i)
-    if (t[i].bn == bn) return &t[i];
+    if (t[i].bn == bn && (ctas == 0 || t[i].ctas == ctas)) return &t[i];
   return nullptr;
 }
 
-// Heuristic: estimated time = waves x per-tile cost, where a 128 x BN tile
-// costs BN (tensor-core time) plus a fixed per-tile overhead for the
-// pipeline fill and epilogue; ragged N tiles waste their missing columns.
+static thread_local int t_force_ctas = 0;
+
+// Heuristic: estimated time = waves x K blocks x cycles per K block (+ a
+// per-tile epilogue term when the accumulator is single-buffered).  Per K
+// block an SM needs 2*BN tensor-core cycles (128 x BN x 128 FP8 MACs at 8192
+// MACs/cycle) and must receive 16 KB of A plus 128*BN/CTAS bytes of B; the
+// operand rate an SM sustains is taken as 64 B/cycle.
 template <int MODE>
-static const Config* choose_config(long long m_tiles_est, int N, int sms) {
-  if (t_force_bn) return find_config<MODE>(t_force_bn);
+static const Config* choose_config(long long rows_est, int N, int K, int sms) {
+  if (t_force_bn) return find_config<MODE>(t_force_bn, t_force_ctas);
   int n = 0;
   const Config* t = config_table<MODE>(&n);
   const Config* best = nullptr;
   double best_cost = 1e300;
+  const double kb = K / 128.0;
   for (int i = 0; i < n; ++i) {
-    const int bn = t[i].bn;
-    const long long n_tiles = (N + bn - 1) / bn;
-    const long long tiles = m_tiles_est * n_tiles;
-    const long long waves = (tiles + sms - 1) / sms;
-    const double cost = static_cast<double>(waves) * (bn + 48.0);
-    if (cost < best_cost - 1e-9) {
+    const Config& c = t[i];
+    const long long tile_m = 128LL * c.ctas;
+    const long long m_tiles = (rows_est + tile_m - 1) / tile_m;
+    const long long n_tiles = (N + c.bn - 1) / c.bn;
+    const long long units = std::max(1, sms / c.ctas);
+    const long long waves = (m_tiles * n_tiles + units - 1) / units;
+    const double mma = 2.0 * c.bn;
+    const double load = (16384.0 + 128.0 * c.bn / c.ctas) / 64.0;
+    const double per_tile = kb * std::max(mma, load) + 600.0 + (c.num_acc == 1 ? 4.0 * c.bn : 0.0);
+    const double cost = static_cast<double>(waves) * per_tile;
+    if (cost < best_cost * 0.999) {
       best_cost = cost;
-      best = &t[i];
+      best = &c;
     }
   }
   return best;
@@ -172,11 +198,45 @@ static const Config* choose_config(long long m_tiles_est, int N, int sms) {
 
 static int raster_group(int num_m_blocks) { return std::min(num_m_blocks, 16); }
 
+// Clusters of two CTAs must sit in one GPC, so fewer than sms/2 pairs may be
+// resident at once; a persistent grid larger than that would run a second
+// wave.  Queried once per configuration and device.
+static int max_active_pairs(const Config* cfg, int sms) {
+  static std::mutex mu;
+  static int cache[64][2][8] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
+  const int key = (cfg->bn / 32) % 8;
+  const int slot = cfg->stages > 5;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev][slot][key] == 0) {
+    if (cudaFuncSetAttribute(reinterpret_cast<const void*>(cfg->fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             cfg->smem) != cudaSuccess)
+      return sms / 2;
+    cudaLaunchConfig_t lc = {};
+    cudaLaunchAttribute attr[1];
+    lc.gridDim = dim3(sms / 2 * 2);
+    lc.blockDim = dim3(kThreads);
+    lc.dynamicSmemBytes = cfg->smem;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(cfg->fn), &lc) != cudaSuccess || n <= 0)
+      n = sms / 2;
+    cache[dev][slot][key] = std::min(n, sms / 2);
+  }
+  return cache[dev][slot][key];
+}
+
 template <int MODE>
 static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const GemmArgs& args,
                   cudaStream_t stream) {
   static std::mutex mu;
-  static bool attr_done[16] = {};
+  static bool attr_done[32] = {};
   int idx = 0;
   {
     int n = 0;
@@ -192,44 +252,50 @@ static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const Ge
     }
   }
   cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
   lc.gridDim = dim3(grid);
   lc.blockDim = dim3(kThreads);
   lc.dynamicSmemBytes = cfg->smem;
   lc.stream = stream;
-  DG_CUDA_TRY(cudaLaunchKernelEx(&lc, cfg->fn, maps[0], maps[1], maps[2], maps[3], maps[4], args));
+  if (cfg->ctas == 2) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+  }
+  DG_CUDA_TRY(cudaLaunchKernelEx(&lc, cfg->fn, maps[0], maps[1], maps[2], args));
   return DG_OK;
 }
 
-// Builds the five tensor maps of one call.
-//   A   : [GA][rowsA][K] bytes           box 128 x 128, 128-byte swizzle
-//   B   : [GB][N][K] bytes               box 128 x BN,  128-byte swizzle
-//   SFA : [GA][Kp][align4(rowsA)] int32  box 128 words
-//   SFB : [GB][Kp][align4(Nb)] int32     box 8 words
-//   D   : [GD][rowsD][N] bf16            box 32 x 32,   64-byte swizzle
-static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const int32_t* sfa,
-                      const void* b, const int32_t* sfb, void* d, int rowsA, int GA, int N, int K,
-                      int GB, int rowsD, int GD) {
-  const uint64_t Kp = (K / 128 + 3) / 4;
-  const uint64_t mn4a = (static_cast<uint64_t>(rowsA) + 3) / 4 * 4;
-  const uint64_t nb4 = (static_cast<uint64_t>((N + 127) / 128) + 3) / 4 * 4;
+// Builds the tensor maps of one call.
+//   A : [GA][rowsA][K] bytes    box 128 x 128 (K x rows), 128-byte swizzle
+//   B : [GB][N][K] bytes        box 128 x BN/CTAS,         128-byte swizzle
+//   D : [GD][rowsD][N] bf16     box 32 x 32,               64-byte swizzle
+static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const void* b, void* d,
+                      int rowsA, int GA, int N, int K, int GB, int rowsD, int GD) {
   int r;
   if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, rowsA, GA, K,
                     static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A")))
     return r;
   if ((r = make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K, N, GB, K,
-                    static_cast<uint64_t>(N) * K, 128, cfg->bn, CU_TENSOR_MAP_SWIZZLE_128B, "B")))
+                    static_cast<uint64_t>(N) * K, 128, cfg->bn / cfg->ctas, CU_TENSOR_MAP_SWIZZLE_128B,
+                    "B")))
     return r;
-  if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_INT32, sfa, mn4a, Kp, GA, mn4a * 4,
-                    Kp * mn4a * 4, 128, 1, CU_TENSOR_MAP_SWIZZLE_NONE, "SFA")))
-    return r;
-  if ((r = make_map(&maps[3], CU_TENSOR_MAP_DATA_TYPE_INT32, sfb, nb4, Kp, GB, nb4 * 4,
-                    Kp * nb4 * 4, 8, 1, CU_TENSOR_MAP_SWIZZLE_NONE, "SFB")))
-    return r;
-  if ((r = make_map(&maps[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, rowsD, GD,
+  if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, rowsD, GD,
                     static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(rowsD) * N * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B, "D")))
     return r;
   return DG_OK;
+}
+
+static void fill_scale_args(GemmArgs* args, const int32_t* sfa, const int32_t* sfb, int rowsA, int N, int K) {
+  args->kp = (K / 128 + 3) / 4;
+  args->mn4a = (rowsA + 3) / 4 * 4;
+  args->nb4 = ((N + 127) / 128 + 3) / 4 * 4;
+  args->sfa = reinterpret_cast<const uint32_t*>(sfa);
+  args->sfb = reinterpret_cast<const uint32_t*>(sfb);
 }
 
 static int check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
@@ -242,10 +308,14 @@ static int check_common(const void* a, const int32_t* sfa, const void* b, const 
   return DG_OK;
 }
 
-static int grid_size(int sms, long long tiles) {
+// Persistent grid: one CTA per SM (co-resident pairs for 2-CTA tiles), never
+// more units than tiles.
+static int grid_size(int sms, long long tiles, const Config* cfg) {
   int g = g_num_sms_override > 0 ? std::min(g_num_sms_override, sms) : sms;
-  if (tiles < g) g = static_cast<int>(std::max<long long>(tiles, 1));
-  return g;
+  long long units = g / cfg->ctas;
+  if (cfg->ctas == 2) units = std::min<long long>(units, max_active_pairs(cfg, sms));
+  if (tiles < units) units = std::max<long long>(tiles, 1);
+  return static_cast<int>(units * cfg->ctas);
 }
 
 // ------------------------------------------------------------------ pack kernel
@@ -293,7 +363,7 @@ using namespace dg;
 
 extern "C" {
 
-int dg_get_mk_alignment_for_contiguous_layout(void) { return kBM; }
+int dg_get_mk_alignment_for_contiguous_layout(void) { return 128; }
 
 int64_t dg_packed_sf_words(int mn, int kb) {
   if (mn < 0 || kb < 0) return -1;
@@ -314,36 +384,40 @@ int dg_get_num_sms(void) {
   return g_num_sms_override > 0 ? std::min(g_num_sms_override, di.sms) : di.sms;
 }
 
-int dg_set_config(int block_n, int stages) {
+int dg_set_config(int block_n, int ctas) {
   if (block_n == 0) {
     t_force_bn = 0;
+    t_force_ctas = 0;
     return DG_OK;
   }
-  if (!find_config<MODE_DENSE>(block_n)) return fail(DG_ERR_UNSUPPORTED, "block_n=%d is not built", block_n);
-  if (stages != 0 && stages != find_config<MODE_DENSE>(block_n)->stages)
-    return fail(DG_ERR_UNSUPPORTED, "block_n=%d is built with %d stages only", block_n,
-                find_config<MODE_DENSE>(block_n)->stages);
+  if (ctas < 0 || ctas > 2) return fail(DG_ERR_UNSUPPORTED, "ctas=%d must be 0, 1 or 2", ctas);
+  if (!find_config<MODE_DENSE>(block_n, ctas))
+    return fail(DG_ERR_UNSUPPORTED, "block_n=%d with ctas=%d is not built", block_n, ctas);
   t_force_bn = block_n;
+  t_force_ctas = ctas;
   return DG_OK;
 }
 
 int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf, int buflen) {
-  (void)K;
   if (!buf || buflen <= 0) return fail(DG_ERR_NULL, "buf must be non-NULL");
   DeviceInfo di;
   int sms = 148;
   if (device_info(&di) == DG_OK) sms = di.sms;
   if (g_num_sms_override > 0) sms = std::min(sms, g_num_sms_override);
-  if (N <= 0) return fail(DG_ERR_SHAPE, "N must be positive");
-  long long mt;
-  if (kind == 2) mt = static_cast<long long>(num_groups) * ((M + kBM - 1) / kBM);
-  else mt = (M + kBM - 1) / kBM;
-  const Config* c = kind == 1 ? choose_config<MODE_CONTIG>(mt, N, sms)
-                    : kind == 2 ? choose_config<MODE_MASKED>(mt, N, sms)
-                                : choose_config<MODE_DENSE>(mt, N, sms);
+  if (N <= 0 || K <= 0) return fail(DG_ERR_SHAPE, "N and K must be positive");
+  const Config* c = nullptr;
+  long long tiles = 0;
+  if (kind == 2) {
+    const long long est = std::max<long long>(1, static_cast<long long>(num_groups) * M / 2);
+    c = choose_config<MODE_MASKED>(est, N, K, sms);
+    if (c) tiles = static_cast<long long>(num_groups) * ((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
+  } else {
+    c = kind == 1 ? choose_config<MODE_CONTIG>(M, N, K, sms) : choose_config<MODE_DENSE>(M, N, K, sms);
+    if (c) tiles = static_cast<long long>((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
+  }
   if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
-  const long long tiles = mt * ((N + c->bn - 1) / c->bn);
-  snprintf(buf, buflen, "%dx%dx%d/%d", kBM, c->bn, c->stages, grid_size(sms, tiles));
+  snprintf(buf, buflen, "%dx%dx%d%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
+           grid_size(sms, tiles, c));
   return DG_OK;
 }
 
@@ -386,22 +460,23 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
   if (M == 0) return DG_OK;
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const int mt = (M + kBM - 1) / kBM;
-  const Config* cfg = choose_config<MODE_DENSE>(mt, N, di.sms);
+  const Config* cfg = choose_config<MODE_DENSE>(M, N, K, di.sms);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
-  CUtensorMap maps[5];
-  if ((r = build_maps(maps, cfg, a, sfa, b, sfb, d, M, 1, N, K, 1, M, 1))) return r;
+  CUtensorMap maps[3];
+  if ((r = build_maps(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1))) return r;
   GemmArgs args = {};
   args.rows = M;
   args.N = N;
   args.K = K;
   args.G = 1;
-  args.num_m_blocks = mt;
+  args.num_m_blocks = (M + 128 * cfg->ctas - 1) / (128 * cfg->ctas);
   args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
-  args.raster_m = raster_group(mt);
+  args.raster_m = raster_group(args.num_m_blocks);
   args.d = static_cast<__nv_bfloat16*>(d);
-  const long long tiles = static_cast<long long>(mt) * args.num_n_blocks;
-  return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles), maps, args, static_cast<cudaStream_t>(stream));
+  fill_scale_args(&args, sfa, sfb, M, N, K);
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles, cfg), maps, args,
+                            static_cast<cudaStream_t>(stream));
 }
 
 int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
@@ -411,28 +486,29 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const
   if (r) return r;
   if (!m_indices) return fail(DG_ERR_NULL, "m_indices must be non-NULL");
   if (num_groups <= 0) return fail(DG_ERR_SHAPE, "num_groups=%d must be positive", num_groups);
-  if (M_total < 0 || M_total % kBM != 0)
-    return fail(DG_ERR_SHAPE, "M_total=%d must be a non-negative multiple of %d", M_total, kBM);
+  if (M_total < 0 || M_total % 128 != 0)
+    return fail(DG_ERR_SHAPE, "M_total=%d must be a non-negative multiple of %d", M_total, 128);
   if (M_total == 0) return DG_OK;
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const int mt = M_total / kBM;
-  const Config* cfg = choose_config<MODE_CONTIG>(mt, N, di.sms);
+  const Config* cfg = choose_config<MODE_CONTIG>(M_total, N, K, di.sms);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
-  CUtensorMap maps[5];
-  if ((r = build_maps(maps, cfg, a, sfa, b, sfb, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
+  CUtensorMap maps[3];
+  if ((r = build_maps(maps, cfg, a, b, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
   GemmArgs args = {};
   args.rows = M_total;
   args.N = N;
   args.K = K;
   args.G = num_groups;
-  args.num_m_blocks = mt;
+  args.num_m_blocks = M_total / 128;
   args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
-  args.raster_m = raster_group(mt);
+  args.raster_m = raster_group(args.num_m_blocks);
   args.m_indices = m_indices;
   args.d = static_cast<__nv_bfloat16*>(d);
-  const long long tiles = static_cast<long long>(mt) * args.num_n_blocks;
-  return launch<MODE_CONTIG>(cfg, grid_size(di.sms, tiles), maps, args, static_cast<cudaStream_t>(stream));
+  fill_scale_args(&args, sfa, sfb, M_total, N, K);
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  return launch<MODE_CONTIG>(cfg, grid_size(di.sms, tiles, cfg), maps, args,
+                             static_cast<cudaStream_t>(stream));
 }
 
 int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
@@ -447,27 +523,27 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const voi
   if (M_max == 0) return DG_OK;
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const int mt_per = (M_max + kBM - 1) / kBM;
   // the device decides the real tile count; the heuristic assumes half-full experts
-  const long long mt_est = std::max<long long>(1, static_cast<long long>(num_groups) * mt_per / 2);
-  const Config* cfg = choose_config<MODE_MASKED>(mt_est, N, di.sms);
+  const long long rows_est = std::max<long long>(1, static_cast<long long>(num_groups) * M_max / 2);
+  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, di.sms);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
-  CUtensorMap maps[5];
-  if ((r = build_maps(maps, cfg, a, sfa, b, sfb, d, M_max, num_groups, N, K, num_groups, M_max,
-                      num_groups)))
+  CUtensorMap maps[3];
+  if ((r = build_maps(maps, cfg, a, b, d, M_max, num_groups, N, K, num_groups, M_max, num_groups)))
     return r;
   GemmArgs args = {};
   args.rows = M_max;
   args.N = N;
   args.K = K;
   args.G = num_groups;
-  args.num_m_blocks = mt_per;
+  args.num_m_blocks = (M_max + 128 * cfg->ctas - 1) / (128 * cfg->ctas);
   args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
   args.raster_m = 1;
   args.masked_m = masked_m;
   args.d = static_cast<__nv_bfloat16*>(d);
-  const long long max_tiles = static_cast<long long>(num_groups) * mt_per * args.num_n_blocks;
-  return launch<MODE_MASKED>(cfg, grid_size(di.sms, max_tiles), maps, args, static_cast<cudaStream_t>(stream));
+  fill_scale_args(&args, sfa, sfb, M_max, N, K);
+  const long long max_tiles = static_cast<long long>(num_groups) * args.num_m_blocks * args.num_n_blocks;
+  return launch<MODE_MASKED>(cfg, grid_size(di.sms, max_tiles, cfg), maps, args,
+                             static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

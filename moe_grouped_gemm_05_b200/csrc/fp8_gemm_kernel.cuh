@@ -14,15 +14,24 @@
 // row (A) and one per column (B), which is exactly the 1x128 / 128x128
 // recipe; the scales are powers of two, so the scaling itself is exact.
 //
-// Roles (one CTA per SM, persistent over output tiles of 128 x BN):
-//   warp 0     TMA producer: A/B K-blocks (+ raw packed scale words every 4
-//              K-blocks) into a STAGES-deep shared-memory ring.
-//   warp 1     TMEM owner and MMA issuer: rearranges the scale words into
-//              the tensor-memory scale layout (tcgen05.cp), issues the MMAs,
-//              commits stage releases and finished accumulators.
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator, BF16 RNE conversion,
+// CTAS = 1: one CTA computes a 128 x BN tile.  CTAS = 2: a cluster of two CTAs
+// computes a 256 x BN tile with tcgen05 cta_group::2 MMAs issued by the first
+// CTA; each CTA loads its own 128 rows of A and BN/2 rows of B, so every SM
+// fetches half of the B tile it would need alone.  No load is multicast.
+//
+// Roles (one CTA per SM, persistent over output tiles):
+//   warp 0     producer: TMA loads of A/B K-blocks into a STAGES-deep ring.
+//   warp 1     TMEM owner; in the first CTA of a pair also the MMA issuer:
+//              tcgen05.cp of the scales, tcgen05.mma, commits of stage
+//              releases and finished accumulators (to both CTAs of a pair).
+//   warps 2-5  epilogue: tcgen05.ld of this CTA's accumulator rows, BF16 RNE,
 //              swizzled staging + TMA store for fully valid 32-row slices,
 //              predicated stores for slices holding padding/masked rows.
+//   warp 6     scale producer: for every group of 4 K-blocks, the packed UE8M0
+//              words of the tile, rearranged into the tensor-memory scale
+//              layout (row/column j of a 128-group at lane j%32, column j/32),
+//              into a kSfStages-deep ring of its own, so the load latency of
+//              the words never sits on the TMA issue path.
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of
 // tile i overlaps the MMAs of tile i+1.
 #pragma once
@@ -38,53 +47,60 @@ __device__ int g_dg_error = 0;
 
 enum : int { MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2 };
 
-constexpr int kBM = 128;
 constexpr int kBK = 128;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
+constexpr int kSfStages = 4;  // scale-word ring depth (groups of 4 K-blocks)
 constexpr int kMaxMaskedGroups = 512;
+constexpr int kMaxSmem = 232448;                  // opt-in shared memory per block on sm_100
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
 
 struct GemmArgs {
   int rows;           // dense: M; contiguous: M_total; masked: M_max
   int N, K, G;
-  int num_m_blocks;   // dense / contiguous
+  int num_m_blocks;   // dense / contiguous, in tiles of 128 * CTAS rows
   int num_n_blocks;
   int raster_m;       // rasterisation group height in M blocks
+  int kp;             // words of packed scales along K: ceil(K/128/4)
+  int mn4a;           // words of packed A scales along M: align4(rows)
+  int nb4;            // words of packed B scales along N: align4(ceil(N/128))
+  const uint32_t* sfa;
+  const uint32_t* sfb;
   const int32_t* m_indices;
   const int32_t* masked_m;
   __nv_bfloat16* d;
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int CTAS>
 struct Layout {
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN must be a multiple of 32 in [32, 256]");
-  static constexpr int kNB128 = (BN + 127) / 128;        // 128-column groups of B scales
-  static constexpr int kABytes = kBM * kBK;              // 16 KB
-  static constexpr int kBBytes = BN * kBK;
-  static constexpr int kSfaRawBytes = 512;               // 128 words
-  static constexpr int kSfbRawBytes = 32;                // 8 words
-  static constexpr int kSfRawStride = 640;
-  static constexpr int kSftABytes = 512;                 // 32 rows x 16 B
-  static constexpr int kSftBBytes = 512 * kNB128;
-  static constexpr int kSftSlot = kSftABytes + kSftBBytes;
-  static constexpr int kEpiBuf = 32 * 32 * 2;            // 32 rows x 32 bf16
+  static_assert(CTAS == 1 || CTAS == 2, "CTAS is 1 or 2");
+  static_assert(BN % 32 == 0 && (BN / CTAS) % 16 == 0 && BN >= 32 && BN <= 256,
+                "BN must be a multiple of 32 in [32, 256] with BN/CTAS a multiple of 16");
+  static constexpr int kTileM = 128 * CTAS;
+  static constexpr int kBRows = BN / CTAS;              // rows of B loaded by each CTA
+  static constexpr int kNB128 = (BN + 127) / 128;       // 128-column groups of B scales
+  static constexpr int kABytes = 128 * kBK;             // 16 KB
+  static constexpr int kBBytes = kBRows * kBK;
+  static constexpr int kSftABytes = 512;                // 32 lanes x 16 B
+  static constexpr int kSftBytes = kSftABytes + 512 * kNB128;
+  static constexpr int kEpiBuf = 32 * 32 * 2;           // 32 rows x 32 bf16
   // TMEM columns: accumulators, then two scale slots of 16 columns (SFA at +0, SFB at +8).
   static constexpr int kSfSlotCols = 16;
-  static constexpr int kAccStride = BN <= 128 ? 128 : 256;  // accumulator buffers start on 128-column bounds
+  static constexpr int kAccStride = BN <= 128 ? 128 : 256;
   static constexpr int kNumAcc = (kAccStride + BN + 2 * kSfSlotCols <= 512) ? 2 : 1;
   static constexpr int kSfBaseCol = (kNumAcc - 1) * kAccStride + ((BN + 15) / 16) * 16;
   static constexpr int kTmemCols = 512;
   // shared-memory offsets (from a 1024-byte aligned base)
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
-  static constexpr int kOffSfRaw = kOffB + STAGES * kBBytes;
-  static constexpr int kOffSft = kOffSfRaw + STAGES * kSfRawStride;
-  static constexpr int kOffEpi = ((kOffSft + 2 * kSftSlot + 1023) / 1024) * 1024;
+  static constexpr int kOffSft = kOffB + STAGES * kBBytes;
+  static constexpr int kOffEpi = ((kOffSft + kSfStages * kSftBytes + 1023) / 1024) * 1024;
   static constexpr int kOffBar = kOffEpi + 4 * 2 * kEpiBuf;
-  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 1;
+  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 1 + 2 * kSfStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag
   static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
   static constexpr int kSmemBytes = kOffGroups + (2 * kMaxMaskedGroups + 1) * 4 + 1024;
+  static_assert(kSmemBytes <= kMaxSmem, "shared-memory budget exceeded");
+  static_assert(kSfBaseCol + 2 * kSfSlotCols <= kTmemCols, "TMEM budget exceeded");
 };
 
 struct Tile {
@@ -93,13 +109,15 @@ struct Tile {
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting
 // (another role gave up) or this wait exceeded its limit (sets the error word).
+template <bool kCluster>
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto probe = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (probe()) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (probe()) return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       *abort_flag = 1;
@@ -129,7 +147,7 @@ __device__ __forceinline__ int total_tiles(const GemmArgs& p, const int* prefix)
 // Tile order: dense / contiguous use groups of `raster_m` M blocks swept
 // column by column, so concurrently running CTAs share A rows and B columns
 // in L2; masked runs expert by expert, N block by N block, M blocks fastest.
-template <int MODE>
+template <int MODE, int TILE_M>
 __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* prefix,
                                         const int* counts) {
   Tile tl;
@@ -137,7 +155,7 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
     int g = 0;
     while (prefix[g + 1] <= t) ++g;
     const int local = t - prefix[g];
-    const int cnt = (counts[g] + kBM - 1) / kBM;
+    const int cnt = (counts[g] + TILE_M - 1) / TILE_M;
     tl.g = g;
     tl.n_blk = local / cnt;
     tl.m_blk = local - tl.n_blk * cnt;
@@ -154,13 +172,12 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
   return tl;
 }
 
-template <int BN, int STAGES, int MODE>
+template <int BN, int STAGES, int MODE, int CTAS>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
-                    const __grid_constant__ CUtensorMap tm_sfa,
-                    const __grid_constant__ CUtensorMap tm_sfb,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
-  using L = Layout<BN, STAGES>;
+  using L = Layout<BN, STAGES, CTAS>;
+  constexpr bool kPair = CTAS == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -171,6 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tmem_empty = bars + 2 * STAGES + 2;
   uint64_t* sf_free = bars + 2 * STAGES + 4;
   uint64_t* final_bar = bars + 2 * STAGES + 6;
+  uint64_t* sf_full = bars + 2 * STAGES + 7;
+  uint64_t* sf_empty = sf_full + kSfStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int* prefix = reinterpret_cast<int*>(smem + L::kOffGroups);
@@ -179,30 +198,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x / 32;
   const int lane = threadIdx.x % 32;
   const int num_kb = p.K / kBK;
+  const uint32_t rank = kPair ? cluster_cta_rank() : 0;
+  const int unit0 = kPair ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
+  const int units = kPair ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full_bar[s], 1);
+      mbar_init(&full_bar[s], CTAS);
       mbar_init(&empty_bar[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tmem_full[i], 1);
-      mbar_init(&tmem_empty[i], 4);
+      mbar_init(&tmem_empty[i], 4 * CTAS);
       mbar_init(&sf_free[i], 1);
     }
     mbar_init(final_bar, 1);
+    for (int i = 0; i < kSfStages; ++i) {
+      mbar_init(&sf_full[i], CTAS);
+      mbar_init(&sf_empty[i], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
-    prefetch_tensormap(&tm_sfa);
-    prefetch_tensormap(&tm_sfb);
     prefetch_tensormap(&tm_d);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, L::kTmemCols);
-    tmem_relinquish();
+    tmem_alloc<CTAS>(tmem_holder, L::kTmemCols);
+    tmem_relinquish<CTAS>();
   }
   if (MODE == MODE_MASKED && warp == 2) {
     // counts[g] = clamp(masked_m[g], 0, M_max); prefix = running sum of tiles
@@ -217,7 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mg = mg < 0 ? 0 : p.rows;
         }
         counts[g] = mg;
-        tiles = ((mg + kBM - 1) / kBM) * p.num_n_blocks;
+        tiles = ((mg + L::kTileM - 1) / L::kTileM) * p.num_n_blocks;
       }
       int incl = tiles;
 #pragma unroll
@@ -231,166 +255,217 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) prefix[0] = 0;
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int ntiles = total_tiles<MODE>(p, prefix);
 
   if (warp == 0) {
     // ============================================================ producer
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-        const Tile tl = tile_of<MODE>(t, p, prefix, counts);
-        int grp_a = 0, grp_b = 0;
-        if (MODE == MODE_CONTIG) {
-          const int e = __ldg(&p.m_indices[tl.m_blk * kBM]);
-          if (e < 0 || e >= p.G) continue;
-          grp_b = e;
-        } else if (MODE == MODE_MASKED) {
-          grp_a = grp_b = tl.g;
-        }
-        const int m0 = tl.m_blk * kBM;
-        const int n0 = tl.n_blk * BN;
-        const int sfb_x = (n0 / 128) & ~3;
-        bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = it % STAGES;
-          if (!wait_phase(&empty_bar[s], ((it / STAGES) & 1) ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const bool with_sf = (kb & 3) == 0;
-          mbar_arrive_expect_tx(&full_bar[s], L::kABytes + L::kBBytes +
-                                                  (with_sf ? L::kSfaRawBytes + L::kSfbRawBytes : 0));
-          tma_load_3d(smem + L::kOffA + s * L::kABytes, &tm_a, &full_bar[s], kb * kBK, m0, grp_a);
-          tma_load_3d(smem + L::kOffB + s * L::kBBytes, &tm_b, &full_bar[s], kb * kBK, n0, grp_b);
-          if (with_sf) {
-            uint8_t* raw = smem + L::kOffSfRaw + s * L::kSfRawStride;
-            tma_load_3d(raw, &tm_sfa, &full_bar[s], m0, kb / 4, grp_a);
-            tma_load_3d(raw + L::kSfaRawBytes, &tm_sfb, &full_bar[s], sfb_x, kb / 4, grp_b);
-          }
-        }
-        if (!ok) break;
+    // Barrier of stage s in the MMA-issuing CTA, as a shared::cluster address.
+    const uint32_t full0 = kPair ? mapa_shared(smem_u32(full_bar), 0) : smem_u32(full_bar);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = unit0; t < ntiles && ok; t += units) {
+      const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
+      int grp_a = 0, grp_b = 0;
+      if (MODE == MODE_CONTIG) {
+        const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
+        if (e < 0 || e >= p.G) continue;
+        grp_b = e;
+      } else if (MODE == MODE_MASKED) {
+        grp_a = grp_b = tl.g;
       }
-      // Drain: every load issued must have landed before the CTA may exit.
+      const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
+      const int n0 = tl.n_blk * BN;
+      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+        const int s = it % STAGES;
+        ok = wait_phase<false>(&empty_bar[s], ((it / STAGES) & 1) ^ 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        if (lane == 0) {
+          uint8_t* a_dst = smem + L::kOffA + s * L::kABytes;
+          uint8_t* b_dst = smem + L::kOffB + s * L::kBBytes;
+          const int b_row = n0 + static_cast<int>(rank) * L::kBRows;
+          if constexpr (kPair) {
+            tma_load_3d_pair(a_dst, &tm_a, full0 + 8 * s, kb * kBK, m_base, grp_a);
+            tma_load_3d_pair(b_dst, &tm_b, full0 + 8 * s, kb * kBK, b_row, grp_b);
+          } else {
+            tma_load_3d(a_dst, &tm_a, &full_bar[s], kb * kBK, m_base, grp_a);
+            tma_load_3d(b_dst, &tm_b, &full_bar[s], kb * kBK, b_row, grp_b);
+          }
+        }
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_expect_tx_cluster(full0 + 8 * s, L::kABytes + L::kBBytes);
+          else mbar_arrive_expect_tx(&full_bar[s], L::kABytes + L::kBBytes);
+        }
+      }
+    }
+    // Drain: every load this CTA's barriers track must land before the CTA exits.
+    if (lane == 0 && (!kPair || rank == 0)) {
       const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0;
       for (uint32_t i = first; i < it; ++i) wait_phase_drain(&full_bar[i % STAGES], (i / STAGES) & 1);
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    uint32_t it = 0, local_tile = 0, sf_group = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
-      const Tile tl = tile_of<MODE>(t, p, prefix, counts);
-      if (MODE == MODE_CONTIG) {
-        const int e = __ldg(&p.m_indices[tl.m_blk * kBM]);
-        if (e < 0 || e >= p.G) continue;
-      }
-      const int n0 = tl.n_blk * BN;
-      const int sfb_x = (n0 / 128) & ~3;
-      const uint32_t acc = local_tile % L::kNumAcc;
-      const uint32_t acc_use = local_tile / L::kNumAcc;
-      ++local_tile;
-      ok = wait_phase(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
-      uint32_t slot = 0;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const int s = it % STAGES;
-        ok = wait_phase(&full_bar[s], (it / STAGES) & 1, abort_flag);
-        if ((kb & 3) == 0 && ok) {
-          slot = sf_group & 1;
-          const uint32_t use = sf_group >> 1;
-          if (use >= 1) ok = wait_phase(&sf_free[slot], (use - 1) & 1, abort_flag);
+    if (!kPair || rank == 0) {
+      uint32_t it = 0, local_tile = 0, sf_group = 0;
+      bool ok = true;
+      for (int t = unit0; t < ntiles && ok; t += units) {
+        const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
+        if (MODE == MODE_CONTIG) {
+          const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
+          if (e < 0 || e >= p.G) continue;
         }
+        const uint32_t acc = local_tile % L::kNumAcc;
+        const uint32_t acc_use = local_tile / L::kNumAcc;
+        ++local_tile;
+        ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        if ((kb & 3) == 0) {
-          // Rearrange this tile's scale words for the tensor-memory scale layout:
-          // row/column j of a 128-wide group lives at (lane j%32, column j/32).
-          const uint32_t* raw = reinterpret_cast<const uint32_t*>(smem + L::kOffSfRaw + s * L::kSfRawStride);
-          uint8_t* sft = smem + L::kOffSft + slot * L::kSftSlot;
-          uint4 va = make_uint4(raw[lane], raw[32 + lane], raw[64 + lane], raw[96 + lane]);
-          *reinterpret_cast<uint4*>(sft + lane * 16) = va;
-          const uint32_t* rawb = raw + L::kSfaRawBytes / 4;
-#pragma unroll
-          for (int h = 0; h < L::kNB128; ++h) {
-            uint32_t w[4];
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const int j = 128 * h + 32 * c + lane;
-              w[c] = (j < BN) ? rawb[(n0 + j) / 128 - sfb_x] : 0u;
-            }
-            *reinterpret_cast<uint4*>(sft + L::kSftABytes + h * 512 + lane * 16) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+        const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
+        uint32_t slot = 0, ring = 0;
+        for (int kb = 0; kb < num_kb; ++kb, ++it) {
+          const int s = it % STAGES;
+          ok = wait_phase<false>(&full_bar[s], (it / STAGES) & 1, abort_flag);
+          if ((kb & 3) == 0 && ok) {
+            slot = sf_group & 1;
+            ring = sf_group % kSfStages;
+            const uint32_t use = sf_group >> 1;
+            if (use >= 1) ok = wait_phase<false>(&sf_free[slot], (use - 1) & 1, abort_flag);
+            // acquire at cluster scope: pairs with the scale producers' release (their
+            // shared-memory writes are read by tcgen05.cp)
+            if (ok) ok = wait_phase<kPair>(&sf_full[ring], (sf_group / kSfStages) & 1, abort_flag);
+            ++sf_group;
           }
-          fence_proxy_async_smem();
-          __syncwarp();
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          tc_fence_after();
           if (lane == 0) {
             const uint32_t sf_col = tmem_base + L::kSfBaseCol + slot * L::kSfSlotCols;
-            tmem_cp_32x128b_warpx4(sf_col, make_smem_desc(smem_u32(sft), 0, 128, 0));
+            if ((kb & 3) == 0) {
+              const uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
+              tmem_cp_32x128b_warpx4<CTAS>(sf_col, make_smem_desc(smem_u32(sft), 0, 128, 0));
 #pragma unroll
-            for (int h = 0; h < L::kNB128; ++h)
-              tmem_cp_32x128b_warpx4(sf_col + 8 + 4 * h,
-                                     make_smem_desc(smem_u32(sft + L::kSftABytes + h * 512), 0, 128, 0));
-          }
-          ++sf_group;
-        }
-        if (lane == 0) {
-          const uint32_t sf_col = tmem_base + L::kSfBaseCol + slot * L::kSfSlotCols;
-          const uint32_t idesc = make_idesc_mxf8(kBM, BN, kb & 3, kb & 3);
-          const uint64_t a_desc = make_smem_desc(smem_u32(smem + L::kOffA + s * L::kABytes), 16, 1024, 2);
-          const uint64_t b_desc = make_smem_desc(smem_u32(smem + L::kOffB + s * L::kBBytes), 16, 1024, 2);
+              for (int h = 0; h < L::kNB128; ++h)
+                tmem_cp_32x128b_warpx4<CTAS>(
+                    sf_col + 8 + 4 * h, make_smem_desc(smem_u32(sft + L::kSftABytes + h * 512), 0, 128, 0));
+            }
+            const uint32_t idesc = make_idesc_mxf8(L::kTileM, BN, kb & 3, kb & 3);
+            const uint64_t a_desc = make_smem_desc(smem_u32(smem + L::kOffA + s * L::kABytes), 16, 1024, 2);
+            const uint64_t b_desc = make_smem_desc(smem_u32(smem + L::kOffB + s * L::kBBytes), 16, 1024, 2);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) {
-            // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
-            mma_mxf8f6f4(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, sf_col, sf_col + 8,
-                         (kb > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < kBK / 32; ++k) {
+              // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, sf_col, sf_col + 8,
+                                 (kb > 0 || k > 0) ? 1u : 0u);
+            }
+            if constexpr (kPair) tc_commit_pair(&empty_bar[s]);
+            else tc_commit<1>(&empty_bar[s]);
+            if ((kb & 3) == 3 || kb == num_kb - 1) {
+              tc_commit<CTAS>(&sf_free[slot]);
+              if constexpr (kPair) tc_commit_pair(&sf_empty[ring]);
+              else tc_commit<1>(&sf_empty[ring]);
+            }
+            if (kb == num_kb - 1) {
+              if constexpr (kPair) tc_commit_pair(&tmem_full[acc]);
+              else tc_commit<1>(&tmem_full[acc]);
+            }
           }
-          tc_commit(&empty_bar[s]);
-          if ((kb & 3) == 3 || kb == num_kb - 1) tc_commit(&sf_free[slot]);
-          if (kb == num_kb - 1) tc_commit(&tmem_full[acc]);
+          __syncwarp();
         }
+      }
+      // Drain: all MMAs / copies issued by this thread complete before TMEM is freed.
+      if (lane == 0) {
+        tc_commit<CTAS>(final_bar);
+        wait_phase_drain(final_bar, 0);
+      }
+      __syncwarp();
+    }
+  } else if (warp == 6) {
+    // ============================================================ scale producer
+    const uint32_t sf_full0 = kPair ? mapa_shared(smem_u32(sf_full), 0) : smem_u32(sf_full);
+    uint32_t group = 0;
+    bool ok = true;
+    for (int t = unit0; t < ntiles && ok; t += units) {
+      const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
+      int grp_a = 0, grp_b = 0;
+      if (MODE == MODE_CONTIG) {
+        const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
+        if (e < 0 || e >= p.G) continue;
+        grp_b = e;
+      } else if (MODE == MODE_MASKED) {
+        grp_a = grp_b = tl.g;
+      }
+      const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
+      const int n0 = tl.n_blk * BN;
+      for (int kp = 0; kp < p.kp; ++kp, ++group) {
+        const uint32_t ring = group % kSfStages;
+        ok = wait_phase<false>(&sf_empty[ring], ((group / kSfStages) & 1) ^ 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        // lane r gathers rows / columns r, r+32, r+64, r+96 of each 128-group
+        const uint32_t* sfa_row = p.sfa + (static_cast<size_t>(grp_a) * p.kp + kp) * p.mn4a;
+        uint32_t wa[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = m_base + 32 * i + lane;
+          wa[i] = m < p.mn4a ? __ldg(sfa_row + m) : 0u;
+        }
+        const uint32_t* sfb_row = p.sfb + (static_cast<size_t>(grp_b) * p.kp + kp) * p.nb4;
+        uint32_t wb[L::kNB128][4];
+#pragma unroll
+        for (int h = 0; h < L::kNB128; ++h)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int j = 128 * h + 32 * c + lane;
+            const int nb = (n0 + j) >> 7;
+            wb[h][c] = (j < BN && nb < p.nb4) ? __ldg(sfb_row + nb) : 0u;
+          }
+        uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
+        *reinterpret_cast<uint4*>(sft + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+#pragma unroll
+        for (int h = 0; h < L::kNB128; ++h)
+          *reinterpret_cast<uint4*>(sft + L::kSftABytes + h * 512 + lane * 16) =
+              make_uint4(wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
+        fence_proxy_async_smem();
         __syncwarp();
+        if (lane == 0) {
+          // the words are read by the tensor core on behalf of the MMA-issuing CTA
+          if constexpr (kPair) mbar_arrive_cluster(sf_full0 + 8 * ring);
+          else mbar_arrive(&sf_full[ring]);
+        }
       }
     }
-    // Drain: all MMAs / copies issued by this thread complete before TMEM is freed.
-    if (lane == 0) {
-      tc_commit(final_bar);
-      wait_phase_drain(final_bar, 0);
-    }
-    __syncwarp();
   } else {
     // ============================================================ epilogue
     const int q = warp % 4;  // TMEM lane quarter this warp may access
     __nv_bfloat16* epi_base = reinterpret_cast<__nv_bfloat16*>(smem + L::kOffEpi + (warp - 2) * 2 * L::kEpiBuf);
+    const uint32_t empty0 = kPair ? mapa_shared(smem_u32(tmem_empty), 0) : smem_u32(tmem_empty);
     uint32_t local_tile = 0, store_count = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      const Tile tl = tile_of<MODE>(t, p, prefix, counts);
+    for (int t = unit0; t < ntiles; t += units) {
+      const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
       int expert = 0;
       if (MODE == MODE_CONTIG) {
-        expert = __ldg(&p.m_indices[tl.m_blk * kBM]);
+        expert = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
         if (expert < 0 || expert >= p.G) {
-          if (expert < -1 || expert >= p.G) {
-            if (warp == 2 && lane == 0 && tl.n_blk == 0) atomicOr(&g_dg_error, 0x2);
-          }
+          if ((expert < -1 || expert >= p.G) && warp == 2 && lane == 0 && tl.n_blk == 0)
+            atomicOr(&g_dg_error, 0x2);
           continue;
         }
       }
       const uint32_t acc = local_tile % L::kNumAcc;
       const uint32_t acc_use = local_tile / L::kNumAcc;
       ++local_tile;
-      bool ok = wait_phase(&tmem_full[acc], acc_use & 1, abort_flag);
+      bool ok = wait_phase<false>(&tmem_full[acc], acc_use & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
 
-      const int row_in_tile = 32 * q + lane;
-      const int m_local = tl.m_blk * kBM + row_in_tile;  // row inside A / D (per expert for masked)
+      const int row0 = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank) + 32 * q;  // warp's first row
+      const int m_local = row0 + lane;  // row inside A / D (per expert for masked)
       bool valid;
       if (MODE == MODE_DENSE) {
         valid = m_local < p.rows;
@@ -403,11 +478,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         valid = m_local < counts[tl.g];
       }
       const bool all_valid = __all_sync(0xffffffffu, valid);
+      const bool any_valid = __any_sync(0xffffffffu, valid);
       const int n0 = tl.n_blk * BN;
       const int zd = (MODE == MODE_MASKED) ? tl.g : 0;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * L::kAccStride;
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 32 && any_valid; ++c) {
         const int col0 = n0 + 32 * c;
         if (col0 >= p.N) break;
         uint32_t r[32];
@@ -434,7 +510,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tm_d, buf, col0, tl.m_blk * kBM + 32 * q, zd);
+            tma_store_3d(&tm_d, buf, col0, row0, zd);
             bulk_commit_group();
           }
         } else if (valid) {
@@ -449,7 +525,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+      if (lane == 0) {
+        if constexpr (kPair) mbar_arrive_remote(empty0 + 8 * acc);
+        else mbar_arrive(&tmem_empty[acc]);
+      }
     }
     if (lane == 0) bulk_wait_group<0>();
     __syncwarp();
@@ -457,10 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
-  __syncthreads();
+  if constexpr (kPair) cluster_sync(); else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, L::kTmemCols);
+    tmem_dealloc<CTAS>(tmem_base, L::kTmemCols);
   }
 }
 

@@ -77,5 +77,7 @@ def test_pack_argument_errors(lib):
 
 def test_config_override(lib):
     assert lib.dg_set_config(96, 0) == -4
+    assert lib.dg_set_config(128, 3) == -4
     assert lib.dg_set_config(128, 0) == 0
+    assert lib.dg_set_config(224, 2) == 0
     assert lib.dg_set_config(0, 0) == 0

@@ -13,7 +13,8 @@ from helpers import bits, check_close, packed, to_device
 
 pytestmark = pytest.mark.gpu
 
-BUILT_BN = (128, 224, 256)
+BUILT = [(128, 1), (224, 1), (256, 1), (128, 2), (224, 2), (256, 2)]  # (block_n, ctas)
+BUILT_1CTA = [c for c in BUILT if c[1] == 1]
 SENTINEL = 0xDEAD
 
 
@@ -71,27 +72,28 @@ def _run_dense(p, sa=None, sb=None):
     return bits(d)
 
 
-@pytest.mark.parametrize("bn", BUILT_BN)
-def test_dense_small_all_configs(bn):
+@pytest.mark.parametrize("cfg", BUILT)
+def test_dense_small_all_configs(cfg):
     p = synth.WORKLOADS["dense_128x512x512"]()
     sa, sb = packed(p)
-    dg.set_config(bn)
+    dg.set_config(*cfg)
     got = _run_dense(p, sa, sb)
     ref = oracle.fp8_gemm_nt(p.a, sa, p.b, sb, p.M, p.N, p.K)
-    check_close(got, ref, f"dense 128x512x512 BN={bn}")
+    check_close(got, ref, f"dense 128x512x512 cfg={cfg}")
     assert dg.get_device_error() == 0
 
 
-@pytest.mark.parametrize("bn", BUILT_BN)
-@pytest.mark.parametrize("shape", [(200, 336, 384), (1, 16, 128), (129, 272, 640), (300, 1008, 1152)])
-def test_dense_ragged(bn, shape):
+@pytest.mark.parametrize("cfg", BUILT)
+@pytest.mark.parametrize("shape", [(200, 336, 384), (1, 16, 128), (129, 272, 640), (300, 1008, 1152),
+                                   (520, 448, 256)])
+def test_dense_ragged(cfg, shape):
     M, N, K = shape
     p = synth.dense_problem(M, N, K, seed=M * 7 + N + K)
     sa, sb = packed(p)
-    dg.set_config(bn)
+    dg.set_config(*cfg)
     got = _run_dense(p, sa, sb)
     ref = oracle.fp8_gemm_nt(p.a, sa, p.b, sb, M, N, K)
-    check_close(got, ref, f"dense {shape} BN={bn}")
+    check_close(got, ref, f"dense {shape} cfg={cfg}")
 
 
 def test_dense_integer_inputs_bit_exact():
@@ -104,11 +106,11 @@ def test_dense_integer_inputs_bit_exact():
     p = synth.Problem("dense", "int", a, np.ones((M, K // 128), np.float32), b,
                       np.ones((N // 128, K // 128), np.float32), M, N, K)
     sa, sb = packed(p)
-    for bn in BUILT_BN:
-        dg.set_config(bn)
+    for cfg in BUILT:
+        dg.set_config(*cfg)
         got = _run_dense(p, sa, sb)
         ref = oracle.fp8_gemm_nt(a, sa, b, sb, M, N, K)
-        assert np.array_equal(got, ref), f"BN={bn}"
+        assert np.array_equal(got, ref), f"cfg={cfg}"
 
 
 def test_dense_all_ones_closed_form():
@@ -122,8 +124,9 @@ def test_dense_all_ones_closed_form():
     assert (got == 0x4400).all()  # 1024 * 2^-3 * 2^2 = 512
 
 
+@pytest.mark.parametrize("cfg", BUILT)
 @pytest.mark.parametrize("lo,hi,exact", [(124, 131, True), (112, 143, False)])
-def test_dense_per_block_scales(lo, hi, exact):
+def test_dense_per_block_scales(cfg, lo, hi, exact):
     # all-ones operands, scales varying per row / per K block / per 128-column block.
     # With exponents in [124, 130] every block term is 128 * 2^[-6, 6] and the FP32
     # sum of eight of them is exact, so the result must match bit for bit; a wide
@@ -135,6 +138,7 @@ def test_dense_per_block_scales(lo, hi, exact):
     p = synth.Problem("dense", "blk", np.full((M, K), 0x38, np.uint8), np.ldexp(1.0, ea - 127).astype(np.float32),
                       np.full((N, K), 0x38, np.uint8), np.ldexp(1.0, eb - 127).astype(np.float32), M, N, K)
     sa, sb = packed(p)
+    dg.set_config(*cfg)
     got = _run_dense(p, sa, sb)
     ref = oracle.fp8_gemm_nt(p.a, sa, p.b, sb, M, N, K)
     if exact:
@@ -146,19 +150,19 @@ def test_dense_per_block_scales(lo, hi, exact):
 # ------------------------------------------------------------------ contiguous
 
 
-@pytest.mark.parametrize("bn", BUILT_BN)
-def test_contiguous_small(bn):
+@pytest.mark.parametrize("cfg", BUILT_1CTA)
+def test_contiguous_small(cfg):
     p = synth.contiguous_problem(4, 512, 512, rows=0, seed=77, counts=[130, 0, 70, 250])
     sa, sb = packed(p)
     t = to_device(p, sa, sb)
-    dg.set_config(bn)
+    dg.set_config(*cfg)
     d = _sentinel((p.M, p.N))
     dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], t["m_indices"], d)
     got = bits(d)
     ref = np.full((p.M, p.N), SENTINEL, np.uint16)
     assert oracle.m_grouped_fp8_gemm_nt_contiguous(p.a, sa, p.b, sb, p.m_indices, ref, p.G, p.N, p.K) == 0
     valid = p.m_indices >= 0
-    check_close(got[valid], ref[valid], f"contiguous BN={bn}")
+    check_close(got[valid], ref[valid], f"contiguous cfg={cfg}")
     assert (got[~valid] == SENTINEL).all()
     assert dg.get_device_error() == 0
 
@@ -186,12 +190,12 @@ def test_contiguous_bad_expert_index_flags_and_skips():
 # ------------------------------------------------------------------ masked
 
 
-@pytest.mark.parametrize("bn", BUILT_BN)
-def test_masked_small(bn):
+@pytest.mark.parametrize("cfg", BUILT)
+def test_masked_small(cfg):
     p = synth.masked_problem(5, 256, 384, 640, seed=91, masked_m=[0, 256, 129, 7, 128])
     sa, sb = packed(p)
     t = to_device(p, sa, sb)
-    dg.set_config(bn)
+    dg.set_config(*cfg)
     d = _sentinel((p.G, p.M, p.N))
     dg.m_grouped_fp8_gemm_nt_masked(t["a"], t["sfa"], t["b"], t["sfb"], t["masked_m"], d)
     got = bits(d)
@@ -199,7 +203,7 @@ def test_masked_small(bn):
     assert oracle.m_grouped_fp8_gemm_nt_masked(p.a, sa, p.b, sb, p.masked_m, ref, p.G, p.M, p.N, p.K) == 0
     for g, mg in enumerate(p.masked_m):
         assert (got[g, mg:] == SENTINEL).all(), f"expert {g}: rows >= {mg} were written"
-        check_close(got[g, :mg], ref[g, :mg], f"masked expert {g} BN={bn}")
+        check_close(got[g, :mg], ref[g, :mg], f"masked expert {g} cfg={cfg}")
     assert dg.get_device_error() == 0
 
 
