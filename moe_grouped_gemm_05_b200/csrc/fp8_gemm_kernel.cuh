@@ -95,7 +95,7 @@ struct Layout {
   static constexpr int kOffSft = kOffB + STAGES * kBBytes;
   static constexpr int kOffEpi = ((kOffSft + kSfStages * kSftBytes + 1023) / 1024) * 1024;
   static constexpr int kOffBar = kOffEpi + 4 * 2 * kEpiBuf;
-  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 1 + 2 * kSfStages;
+  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 1 + 2 * kSfStages;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag
   static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
   static constexpr int kSmemBytes = kOffGroups + (2 * kMaxMaskedGroups + 1) * 4 + 1024;
@@ -186,9 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tmem_full = bars + 2 * STAGES;
   uint64_t* tmem_empty = bars + 2 * STAGES + 2;
-  uint64_t* sf_free = bars + 2 * STAGES + 4;
-  uint64_t* final_bar = bars + 2 * STAGES + 6;
-  uint64_t* sf_full = bars + 2 * STAGES + 7;
+  uint64_t* final_bar = bars + 2 * STAGES + 4;
+  uint64_t* sf_full = bars + 2 * STAGES + 5;
   uint64_t* sf_empty = sf_full + kSfStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
@@ -211,7 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tmem_full[i], 1);
       mbar_init(&tmem_empty[i], 4 * CTAS);
-      mbar_init(&sf_free[i], 1);
     }
     mbar_init(final_bar, 1);
     for (int i = 0; i < kSfStages; ++i) {
@@ -309,8 +307,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ============================================================ MMA issuer
-    if (!kPair || rank == 0) {
-      uint32_t it = 0, local_tile = 0, sf_group = 0;
+    // A single thread issues.  Each tcgen05 instruction costs the issuing
+    // thread ~60 cycles, close to the tensor-pipe time of a K=32 MMA, so the
+    // loop keeps everything else off the per-K-block path: descriptors and
+    // instruction words are precomputed, stage/phase counters are
+    // incremental, barrier polls take an inline fast path, and the only
+    // per-K-block instructions are the wait, four MMAs and one commit.
+    if ((!kPair || rank == 0) && lane == 0) {
+      const uint64_t a_desc0 = make_smem_desc(smem_u32(smem + L::kOffA), 16, 1024, 2);
+      const uint64_t b_desc0 = make_smem_desc(smem_u32(smem + L::kOffB), 16, 1024, 2);
+      uint32_t idesc[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) idesc[j] = make_idesc_mxf8(L::kTileM, BN, j, j);
+      uint32_t s = 0, phase = 0, local_tile = 0, sf_group = 0;
       bool ok = true;
       for (int t = unit0; t < ntiles && ok; t += units) {
         const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
@@ -321,69 +330,67 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t acc = local_tile % L::kNumAcc;
         const uint32_t acc_use = local_tile / L::kNumAcc;
         ++local_tile;
-        ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
-        ok = __all_sync(0xffffffffu, ok);
+        if (!mbar_try_wait(&tmem_empty[acc], (acc_use & 1) ^ 1))
+          ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
-        uint32_t slot = 0, ring = 0;
-        for (int kb = 0; kb < num_kb; ++kb, ++it) {
-          const int s = it % STAGES;
-          ok = wait_phase<false>(&full_bar[s], (it / STAGES) & 1, abort_flag);
-          if ((kb & 3) == 0 && ok) {
-            slot = sf_group & 1;
+        uint32_t sf_col = 0, ring = 0;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if ((kb & 3) == 0) {
             ring = sf_group % kSfStages;
-            const uint32_t use = sf_group >> 1;
-            if (use >= 1) ok = wait_phase<false>(&sf_free[slot], (use - 1) & 1, abort_flag);
+            sf_col = tmem_base + L::kSfBaseCol + (sf_group & 1) * L::kSfSlotCols;
+            // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
+            if (sf_group >= 2) {
+              uint64_t* b = &sf_empty[(sf_group - 2) % kSfStages];
+              const uint32_t par = ((sf_group - 2) / kSfStages) & 1;
+              if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag);
+            }
             // acquire at cluster scope: pairs with the scale producers' release (their
             // shared-memory writes are read by tcgen05.cp)
             if (ok) ok = wait_phase<kPair>(&sf_full[ring], (sf_group / kSfStages) & 1, abort_flag);
             ++sf_group;
-          }
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-          if (lane == 0) {
-            const uint32_t sf_col = tmem_base + L::kSfBaseCol + slot * L::kSfSlotCols;
-            if ((kb & 3) == 0) {
-              const uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
-              tmem_cp_32x128b_warpx4<CTAS>(sf_col, make_smem_desc(smem_u32(sft), 0, 128, 0));
+            if (!ok) break;
+            tc_fence_after();
+            const uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
+            tmem_cp_32x128b_warpx4<CTAS>(sf_col, make_smem_desc(smem_u32(sft), 0, 128, 0));
 #pragma unroll
-              for (int h = 0; h < L::kNB128; ++h)
-                tmem_cp_32x128b_warpx4<CTAS>(
-                    sf_col + 8 + 4 * h, make_smem_desc(smem_u32(sft + L::kSftABytes + h * 512), 0, 128, 0));
-            }
-            const uint32_t idesc = make_idesc_mxf8(L::kTileM, BN, kb & 3, kb & 3);
-            const uint64_t a_desc = make_smem_desc(smem_u32(smem + L::kOffA + s * L::kABytes), 16, 1024, 2);
-            const uint64_t b_desc = make_smem_desc(smem_u32(smem + L::kOffB + s * L::kBBytes), 16, 1024, 2);
-#pragma unroll
-            for (int k = 0; k < kBK / 32; ++k) {
-              // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
-              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2 * k, b_desc + 2 * k, idesc, sf_col, sf_col + 8,
-                                 (kb > 0 || k > 0) ? 1u : 0u);
-            }
-            if constexpr (kPair) tc_commit_pair(&empty_bar[s]);
-            else tc_commit<1>(&empty_bar[s]);
-            if ((kb & 3) == 3 || kb == num_kb - 1) {
-              tc_commit<CTAS>(&sf_free[slot]);
-              if constexpr (kPair) tc_commit_pair(&sf_empty[ring]);
-              else tc_commit<1>(&sf_empty[ring]);
-            }
-            if (kb == num_kb - 1) {
-              if constexpr (kPair) tc_commit_pair(&tmem_full[acc]);
-              else tc_commit<1>(&tmem_full[acc]);
-            }
+            for (int h = 0; h < L::kNB128; ++h)
+              tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8 + 4 * h,
+                                           make_smem_desc(smem_u32(sft + L::kSftABytes + h * 512), 0, 128, 0));
           }
-          __syncwarp();
+          if (!mbar_try_wait(&full_bar[s], phase)) {
+            ok = wait_phase<false>(&full_bar[s], phase, abort_flag);
+            if (!ok) break;
+          }
+          const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (L::kABytes >> 4));
+          const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s * (L::kBBytes >> 4));
+          const uint32_t id = idesc[kb & 3];
+          // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc, b_desc, id, sf_col, sf_col + 8, kb > 0 ? 1u : 0u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2, b_desc + 2, id, sf_col, sf_col + 8, 1u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 4, b_desc + 4, id, sf_col, sf_col + 8, 1u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 6, b_desc + 6, id, sf_col, sf_col + 8, 1u);
+          if constexpr (kPair) tc_commit_pair(&empty_bar[s]);
+          else tc_commit<1>(&empty_bar[s]);
+          if ((kb & 3) == 3 || kb == num_kb - 1) {
+            if constexpr (kPair) tc_commit_pair(&sf_empty[ring]);
+            else tc_commit<1>(&sf_empty[ring]);
+          }
+          if (++s == STAGES) {
+            s = 0;
+            phase ^= 1;
+          }
         }
+        if (!ok) break;
+        if constexpr (kPair) tc_commit_pair(&tmem_full[acc]);
+        else tc_commit<1>(&tmem_full[acc]);
       }
       // Drain: all MMAs / copies issued by this thread complete before TMEM is freed.
-      if (lane == 0) {
-        tc_commit<CTAS>(final_bar);
-        wait_phase_drain(final_bar, 0);
-      }
-      __syncwarp();
+      tc_commit<CTAS>(final_bar);
+      wait_phase_drain(final_bar, 0);
     }
+    __syncwarp();
   } else if (warp == 6) {
     // ============================================================ scale producer
     const uint32_t sf_full0 = kPair ? mapa_shared(smem_u32(sf_full), 0) : smem_u32(sf_full);
