@@ -30,7 +30,7 @@
 //   warp 6     scale producer: for every group of 4 K-blocks, the packed UE8M0
 //              words of the tile, rearranged into the tensor-memory scale
 //              layout (row/column j of a 128-group at lane j%32, column j/32),
-//              into a kSfStages-deep ring of its own, so the load latency of
+//              into a 2- or 4-deep ring of its own, so the load latency of
 //              the words never sits on the TMA issue path.
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of
 // tile i overlaps the MMAs of tile i+1.
@@ -49,7 +49,6 @@ enum : int { MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2 };
 
 constexpr int kBK = 128;
 constexpr int kThreads = 224;
-constexpr int kSfStages = 4;  // scale-word ring depth (groups of 4 K-blocks)
 constexpr int kMaxMaskedGroups = 512;
 constexpr int kMaxSmem = 232448;                  // opt-in shared memory per block on sm_100
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
@@ -80,10 +79,14 @@ struct Layout {
   static constexpr int kNB128 = (BN + 127) / 128;       // 128-column groups of B scales
   static constexpr int kABytes = 128 * kBK;             // 16 KB
   static constexpr int kBBytes = kBRows * kBK;
-  static constexpr int kSftABytes = 512;                // 32 lanes x 16 B
-  static constexpr int kSftBytes = kSftABytes + 512 * kNB128;
+  // Scale words of one K group in shared memory, as tcgen05.cp sources:
+  // 128 rows x 32 B (core-matrix layout) holding [SFA | SFB of columns 0-127]
+  // for TMEM columns +0..+7 (rows r, r+32, r+64, r+96 identical), then, when
+  // BN > 128, 32 rows x 16 B with SFB of columns 128-255 for columns +8..+11.
+  static constexpr int kSftMainBytes = 4096;
+  static constexpr int kSftBytes = kSftMainBytes + (kNB128 == 2 ? 512 : 0);
   static constexpr int kEpiBuf = 32 * 32 * 2;           // 32 rows x 32 bf16
-  // TMEM columns: accumulators, then two scale slots of 16 columns (SFA at +0, SFB at +8).
+  // TMEM columns: accumulators, then two scale slots of 16 columns (SFA at +0, SFB at +4).
   static constexpr int kSfSlotCols = 16;
   static constexpr int kAccStride = BN <= 128 ? 128 : 256;
   static constexpr int kNumAcc = (kAccStride + BN + 2 * kSfSlotCols <= 512) ? 2 : 1;
@@ -93,9 +96,12 @@ struct Layout {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSft = kOffB + STAGES * kBBytes;
-  static constexpr int kOffEpi = ((kOffSft + kSfStages * kSftBytes + 1023) / 1024) * 1024;
+  // scale ring depth: 4 groups when shared memory allows, else 2
+  static constexpr int kSfRing =
+      (kOffSft + 4 * kSftBytes + 1023) / 1024 * 1024 + 4 * 2 * kEpiBuf + 4096 + (2 * kMaxMaskedGroups + 1) * 4 + 1024 <= kMaxSmem ? 4 : 2;
+  static constexpr int kOffEpi = ((kOffSft + kSfRing * kSftBytes + 1023) / 1024) * 1024;
   static constexpr int kOffBar = kOffEpi + 4 * 2 * kEpiBuf;
-  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 1 + 2 * kSfStages;
+  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 1 + 2 * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag
   static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
   static constexpr int kSmemBytes = kOffGroups + (2 * kMaxMaskedGroups + 1) * 4 + 1024;
@@ -188,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tmem_empty = bars + 2 * STAGES + 2;
   uint64_t* final_bar = bars + 2 * STAGES + 4;
   uint64_t* sf_full = bars + 2 * STAGES + 5;
-  uint64_t* sf_empty = sf_full + kSfStages;
+  uint64_t* sf_empty = sf_full + L::kSfRing;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int* prefix = reinterpret_cast<int*>(smem + L::kOffGroups);
@@ -212,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&tmem_empty[i], 4 * CTAS);
     }
     mbar_init(final_bar, 1);
-    for (int i = 0; i < kSfStages; ++i) {
+    for (int i = 0; i < L::kSfRing; ++i) {
       mbar_init(&sf_full[i], CTAS);
       mbar_init(&sf_empty[i], 1);
     }
@@ -338,26 +344,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t sf_col = 0, ring = 0;
         for (int kb = 0; kb < num_kb; ++kb) {
           if ((kb & 3) == 0) {
-            ring = sf_group % kSfStages;
+            ring = sf_group % L::kSfRing;
             sf_col = tmem_base + L::kSfBaseCol + (sf_group & 1) * L::kSfSlotCols;
             // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
             if (sf_group >= 2) {
-              uint64_t* b = &sf_empty[(sf_group - 2) % kSfStages];
-              const uint32_t par = ((sf_group - 2) / kSfStages) & 1;
+              uint64_t* b = &sf_empty[(sf_group - 2) % L::kSfRing];
+              const uint32_t par = ((sf_group - 2) / L::kSfRing) & 1;
               if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag);
             }
             // acquire at cluster scope: pairs with the scale producers' release (their
             // shared-memory writes are read by tcgen05.cp)
-            if (ok) ok = wait_phase<kPair>(&sf_full[ring], (sf_group / kSfStages) & 1, abort_flag);
+            if (ok) ok = wait_phase<kPair>(&sf_full[ring], (sf_group / L::kSfRing) & 1, abort_flag);
             ++sf_group;
             if (!ok) break;
             tc_fence_after();
             const uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
-            tmem_cp_32x128b_warpx4<CTAS>(sf_col, make_smem_desc(smem_u32(sft), 0, 128, 0));
-#pragma unroll
-            for (int h = 0; h < L::kNB128; ++h)
-              tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8 + 4 * h,
-                                           make_smem_desc(smem_u32(sft + L::kSftABytes + h * 512), 0, 128, 0));
+            tmem_cp_128x256b<CTAS>(sf_col, make_smem_desc(smem_u32(sft), 128, 256, 0));
+            if constexpr (L::kNB128 == 2)
+              tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8,
+                                           make_smem_desc(smem_u32(sft + L::kSftMainBytes), 0, 128, 0));
           }
           if (!mbar_try_wait(&full_bar[s], phase)) {
             ok = wait_phase<false>(&full_bar[s], phase, abort_flag);
@@ -367,10 +372,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s * (L::kBBytes >> 4));
           const uint32_t id = idesc[kb & 3];
           // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc, b_desc, id, sf_col, sf_col + 8, kb > 0 ? 1u : 0u);
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2, b_desc + 2, id, sf_col, sf_col + 8, 1u);
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 4, b_desc + 4, id, sf_col, sf_col + 8, 1u);
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 6, b_desc + 6, id, sf_col, sf_col + 8, 1u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc, b_desc, id, sf_col, sf_col + 4, kb > 0 ? 1u : 0u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2, b_desc + 2, id, sf_col, sf_col + 4, 1u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 4, b_desc + 4, id, sf_col, sf_col + 4, 1u);
+          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 6, b_desc + 6, id, sf_col, sf_col + 4, 1u);
           if constexpr (kPair) tc_commit_pair(&empty_bar[s]);
           else tc_commit<1>(&empty_bar[s]);
           if ((kb & 3) == 3 || kb == num_kb - 1) {
@@ -409,8 +414,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
       for (int kp = 0; kp < p.kp; ++kp, ++group) {
-        const uint32_t ring = group % kSfStages;
-        ok = wait_phase<false>(&sf_empty[ring], ((group / kSfStages) & 1) ^ 1, abort_flag);
+        const uint32_t ring = group % L::kSfRing;
+        ok = wait_phase<false>(&sf_empty[ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         // lane r gathers rows / columns r, r+32, r+64, r+96 of each 128-group
@@ -432,11 +437,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             wb[h][c] = (j < BN && nb < p.nb4) ? __ldg(sfb_row + nb) : 0u;
           }
         uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
-        *reinterpret_cast<uint4*>(sft + lane * 16) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        const uint4 va = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        const uint4 vb = make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
 #pragma unroll
-        for (int h = 0; h < L::kNB128; ++h)
-          *reinterpret_cast<uint4*>(sft + L::kSftABytes + h * 512 + lane * 16) =
-              make_uint4(wb[h][0], wb[h][1], wb[h][2], wb[h][3]);
+        for (int q = 0; q < 4; ++q) {  // TMEM lane quarters q hold identical copies
+          const int row = lane + 32 * q;
+          uint8_t* cm = sft + (row >> 3) * 256 + (row & 7) * 16;
+          *reinterpret_cast<uint4*>(cm) = va;         // TMEM columns +0..+3: SFA
+          *reinterpret_cast<uint4*>(cm + 128) = vb;   // TMEM columns +4..+7: SFB, columns 0-127
+        }
+        if constexpr (L::kNB128 == 2)
+          *reinterpret_cast<uint4*>(sft + L::kSftMainBytes + lane * 16) =
+              make_uint4(wb[1][0], wb[1][1], wb[1][2], wb[1][3]);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {

@@ -274,6 +274,18 @@ __device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t 
                  : "memory");
 }
 
+// Copies 128 rows x 256 bits from shared memory into TMEM lanes 0-127, columns
+// [taddr, taddr+8).  The source is described K-major without swizzle: core
+// matrices of 8 rows x 16 bytes, LBO between the two 16-byte halves of a row,
+// SBO between groups of 8 rows.
+template <int CG>
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t sdesc) {
+  if constexpr (CG == 1)
+    asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+  else
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
