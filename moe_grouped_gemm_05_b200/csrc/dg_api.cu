@@ -164,30 +164,41 @@ static const Config* find_config(int bn, int ctas) {
 
 static thread_local int t_force_ctas = 0;
 
-// Heuristic: estimated time = waves x K blocks x cycles per K block (+ a
-// per-tile epilogue term when the accumulator is single-buffered).  Per K
-// block an SM needs 2*BN tensor-core cycles (128 x BN x 128 FP8 MACs at 8192
-// MACs/cycle) and must receive 16 KB of A plus 128*BN/CTAS bytes of B; the
-// operand rate an SM sustains is taken as 64 B/cycle.
+// Heuristic.  Each configuration has a sustained rate measured on B200 with
+// full waves and cold L2 (dense 4096x7168x2048, 8192^3, contiguous and
+// masked workloads, FP8 TFLOP/s): 128-wide tiles run at ~0.62 of the
+// 224/256-wide ones because the per-K-block issue cost of the MMA thread,
+// not the tensor pipe, bounds narrow tiles.  The estimated time of a
+// configuration is its padded work (whole tiles, whole waves of
+// co-resident units) divided by that rate.  The masked layout keeps 1-CTA
+// tiles: a 256-row tile wastes half its work on experts with <= 128 valid
+// rows.
+static double config_rate(const Config& c) {
+  if (c.bn <= 128) return c.ctas == 2 ? 1270.0 : 1290.0;
+  if (c.bn <= 224) return c.ctas == 2 ? 2100.0 : 2050.0;
+  return c.ctas == 2 ? 2150.0 : 2100.0;
+}
+
 template <int MODE>
 static const Config* choose_config(long long rows_est, int N, int K, int sms) {
   if (t_force_bn) return find_config<MODE>(t_force_bn, t_force_ctas);
+  (void)K;
   int n = 0;
   const Config* t = config_table<MODE>(&n);
   const Config* best = nullptr;
   double best_cost = 1e300;
-  const double kb = K / 128.0;
   for (int i = 0; i < n; ++i) {
     const Config& c = t[i];
+    if (MODE == MODE_MASKED && c.ctas != 1) continue;
     const long long tile_m = 128LL * c.ctas;
     const long long m_tiles = (rows_est + tile_m - 1) / tile_m;
     const long long n_tiles = (N + c.bn - 1) / c.bn;
     const long long units = std::max(1, sms / c.ctas);
-    const long long waves = (m_tiles * n_tiles + units - 1) / units;
-    const double mma = 2.0 * c.bn;
-    const double load = (16384.0 + 128.0 * c.bn / c.ctas) / 64.0;
-    const double per_tile = kb * std::max(mma, load) + 600.0 + (c.num_acc == 1 ? 4.0 * c.bn : 0.0);
-    const double cost = static_cast<double>(waves) * per_tile;
+    const long long tiles = m_tiles * n_tiles;
+    const long long waves = (tiles + units - 1) / units;
+    // padded work in units of 128x128 tile-K-blocks, spread over the whole grid
+    const double work = static_cast<double>(waves) * units * (tile_m / 128.0) * (c.bn / 128.0);
+    const double cost = work / config_rate(c);
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = &c;
@@ -287,6 +298,59 @@ static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const
                     static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(rowsD) * N * 2, 32, 32,
                     CU_TENSOR_MAP_SWIZZLE_64B, "D")))
     return r;
+  return DG_OK;
+}
+
+// Tensor maps depend only on pointers, shapes and the tile configuration, so
+// repeated calls (weights, rotating activation buffers, graph replays on the
+// host side) reuse them: a small per-thread direct-mapped cache keyed by all
+// inputs of build_maps.
+struct MapKey {
+  const void* a;
+  const void* b;
+  const void* d;
+  const void* cfg;
+  int rowsA, GA, N, K, GB, rowsD, GD, dev;
+  bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+struct MapEntry {
+  bool valid = false;
+  MapKey key;
+  CUtensorMap maps[3];
+};
+
+static int build_maps_cached(CUtensorMap* maps, const Config* cfg, const void* a, const void* b, void* d,
+                             int rowsA, int GA, int N, int K, int GB, int rowsD, int GD) {
+  constexpr int kSlots = 64;
+  static thread_local MapEntry cache[kSlots];
+  MapKey key;
+  std::memset(&key, 0, sizeof(key));
+  key.a = a;
+  key.b = b;
+  key.d = d;
+  key.cfg = cfg;
+  key.rowsA = rowsA;
+  key.GA = GA;
+  key.N = N;
+  key.K = K;
+  key.GB = GB;
+  key.rowsD = rowsD;
+  key.GD = GD;
+  if (cudaGetDevice(&key.dev) != cudaSuccess) key.dev = -1;
+  uint64_t h = 1469598103934665603ull;
+  const unsigned char* kb = reinterpret_cast<const unsigned char*>(&key);
+  for (size_t i = 0; i < sizeof(key); ++i) h = (h ^ kb[i]) * 1099511628211ull;
+  MapEntry& e = cache[h % kSlots];
+  if (e.valid && e.key == key) {
+    std::memcpy(maps, e.maps, sizeof(e.maps));
+    return DG_OK;
+  }
+  int r = build_maps(maps, cfg, a, b, d, rowsA, GA, N, K, GB, rowsD, GD);
+  if (r) return r;
+  e.valid = true;
+  e.key = key;
+  std::memcpy(e.maps, maps, sizeof(e.maps));
   return DG_OK;
 }
 
@@ -463,7 +527,7 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
   const Config* cfg = choose_config<MODE_DENSE>(M, N, K, di.sms);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
-  if ((r = build_maps(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1))) return r;
+  if ((r = build_maps_cached(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1))) return r;
   GemmArgs args = {};
   args.rows = M;
   args.N = N;
@@ -494,7 +558,7 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const
   const Config* cfg = choose_config<MODE_CONTIG>(M_total, N, K, di.sms);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
-  if ((r = build_maps(maps, cfg, a, b, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
+  if ((r = build_maps_cached(maps, cfg, a, b, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
   GemmArgs args = {};
   args.rows = M_total;
   args.N = N;
@@ -528,7 +592,7 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const voi
   const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, di.sms);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
-  if ((r = build_maps(maps, cfg, a, b, d, M_max, num_groups, N, K, num_groups, M_max, num_groups)))
+  if ((r = build_maps_cached(maps, cfg, a, b, d, M_max, num_groups, N, K, num_groups, M_max, num_groups)))
     return r;
   GemmArgs args = {};
   args.rows = M_max;
