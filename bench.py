@@ -321,7 +321,7 @@ def run_ours(args):
     import torch.distributed as dist
 
     from moe_grouped_gemm_05_b200 import binding as dg
-    from moe_grouped_gemm_05_b200 import synth
+    from moe_grouped_gemm_05_b200 import shard, synth
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -408,10 +408,8 @@ def run_ours(args):
     torch.cuda.synchronize()
     sampler.stop()
     gemm_avg_ms = g0.elapsed_time(g1) / args.steps
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_ms = float(t.item())
+    elapsed_ms = shard.max_over_ranks(elapsed_ms)
+    gemm_avg_ms = shard.max_over_ranks(gemm_avg_ms)
     err = dg.get_device_error()
 
     # end to end through the public API: pinned host inputs in, result out, every step
@@ -442,10 +440,7 @@ def run_ours(args):
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
-    e2e_ms = float(e2e_ms.item())
+    e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1))
 
     flops = p.flops
     value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
