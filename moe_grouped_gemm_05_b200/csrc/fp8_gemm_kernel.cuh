@@ -314,78 +314,92 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ============================================================ MMA issuer
     // A single thread issues.  Each tcgen05 instruction costs the issuing
-    // thread ~60 cycles, close to the tensor-pipe time of a K=32 MMA, so the
-    // loop keeps everything else off the per-K-block path: descriptors and
-    // instruction words are precomputed, stage/phase counters are
-    // incremental, barrier polls take an inline fast path, and the only
-    // per-K-block instructions are the wait, four MMAs and one commit.
+    // thread ~60 cycles and every other instruction a few more, against 448
+    // tensor-pipe cycles per 128x224x128 K block, so the loop is shaped to
+    // execute as little as possible per K block: one iteration covers a whole
+    // scale group (4 K blocks, unrolled), descriptors and instruction words
+    // are precomputed, stage/phase counters are incremental and barrier polls
+    // take an inline fast path.
     if ((!kPair || rank == 0) && lane == 0) {
-      const uint64_t a_desc0 = make_smem_desc(smem_u32(smem + L::kOffA), 16, 1024, 2);
-      const uint64_t b_desc0 = make_smem_desc(smem_u32(smem + L::kOffB), 16, 1024, 2);
-      uint32_t idesc[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) idesc[j] = make_idesc_mxf8(L::kTileM, BN, j, j);
+      const uint32_t a_lo0 = static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffA), 16, 1024, 2));
+      const uint32_t b_lo0 = static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffB), 16, 1024, 2));
+      const uint32_t desc_hi = static_cast<uint32_t>(make_smem_desc(0, 16, 1024, 2) >> 32);
+      const uint32_t idesc0 = make_idesc_mxf8(L::kTileM, BN, 0, 0);
+      constexpr uint32_t kSfIdStep = (1u << 4) | (1u << 29);  // +1 in both scale-factor byte selectors
+      const uint32_t full_base = smem_u32(full_bar);
+      const uint32_t empty_base = smem_u32(empty_bar);
       uint32_t s = 0, phase = 0, local_tile = 0, sf_group = 0;
       bool ok = true;
+      const uint32_t sft_lo0 = static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffSft), 128, 256, 0));
+      const uint32_t sft_hi = static_cast<uint32_t>(make_smem_desc(0, 128, 256, 0) >> 32);
+      const uint32_t sfx_hi = static_cast<uint32_t>(make_smem_desc(0, 0, 128, 0) >> 32);
       for (int t = unit0; t < ntiles && ok; t += units) {
-        const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
-        if (MODE == MODE_CONTIG) {
+        if (MODE == MODE_CONTIG) {  // only the contiguous layout can skip a tile
+          const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
           const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
           if (e < 0 || e >= p.G) continue;
         }
-        const uint32_t acc = local_tile % L::kNumAcc;
-        const uint32_t acc_use = local_tile / L::kNumAcc;
+        const uint32_t acc = L::kNumAcc == 1 ? 0 : (local_tile & 1);
+        const uint32_t acc_use = L::kNumAcc == 1 ? local_tile : (local_tile >> 1);
         ++local_tile;
         if (!mbar_try_wait(&tmem_empty[acc], (acc_use & 1) ^ 1))
           ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
-        uint32_t sf_col = 0, ring = 0;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if ((kb & 3) == 0) {
-            ring = sf_group % L::kSfRing;
-            sf_col = tmem_base + L::kSfBaseCol + (sf_group & 1) * L::kSfSlotCols;
-            // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
-            if (sf_group >= 2) {
-              uint64_t* b = &sf_empty[(sf_group - 2) % L::kSfRing];
-              const uint32_t par = ((sf_group - 2) / L::kSfRing) & 1;
-              if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag);
-            }
-            // acquire at cluster scope: pairs with the scale producers' release (their
-            // shared-memory writes are read by tcgen05.cp)
-            if (ok) ok = wait_phase<kPair>(&sf_full[ring], (sf_group / L::kSfRing) & 1, abort_flag);
-            ++sf_group;
-            if (!ok) break;
-            tc_fence_after();
-            const uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
-            tmem_cp_128x256b<CTAS>(sf_col, make_smem_desc(smem_u32(sft), 128, 256, 0));
+        uint32_t accumulate = 0;
+        for (int kb0 = 0; kb0 < num_kb && ok; kb0 += 4, ++sf_group) {
+          const uint32_t ring = sf_group % L::kSfRing;
+          const uint32_t sf_col = tmem_base + L::kSfBaseCol + (sf_group & 1) * L::kSfSlotCols;
+          // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
+          if (sf_group >= 2) {
+            uint64_t* b = &sf_empty[(sf_group - 2) % L::kSfRing];
+            const uint32_t par = ((sf_group - 2) / L::kSfRing) & 1;
+            if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag);
+          }
+          // acquire at cluster scope: pairs with the scale producers' release (their
+          // shared-memory writes are read by tcgen05.cp)
+          if (ok && !(kPair ? mbar_try_wait_cluster(&sf_full[ring], (sf_group / L::kSfRing) & 1)
+                            : mbar_try_wait(&sf_full[ring], (sf_group / L::kSfRing) & 1)))
+            ok = wait_phase<kPair>(&sf_full[ring], (sf_group / L::kSfRing) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          {
+            const uint32_t lo = sft_lo0 + ring * (L::kSftBytes >> 4);
+            tmem_cp_128x256b<CTAS>(sf_col, (static_cast<uint64_t>(sft_hi) << 32) | lo);
             if constexpr (L::kNB128 == 2)
-              tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8,
-                                           make_smem_desc(smem_u32(sft + L::kSftMainBytes), 0, 128, 0));
+              tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8, (static_cast<uint64_t>(sfx_hi) << 32) |
+                                                           (lo + (L::kSftMainBytes >> 4)));
           }
-          if (!mbar_try_wait(&full_bar[s], phase)) {
-            ok = wait_phase<false>(&full_bar[s], phase, abort_flag);
-            if (!ok) break;
+          const int nk = min(4, num_kb - kb0);
+          uint32_t id = idesc0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              if (!mbar_try_wait_addr(full_base + 8 * s, phase)) {
+                ok = wait_phase<false>(&full_bar[s], phase, abort_flag);
+                if (!ok) break;
+              }
+              const uint64_t a_desc = (static_cast<uint64_t>(desc_hi) << 32) | (a_lo0 + s * (L::kABytes >> 4));
+              const uint64_t b_desc = (static_cast<uint64_t>(desc_hi) << 32) | (b_lo0 + s * (L::kBBytes >> 4));
+              // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc, b_desc, id, sf_col, sf_col + 4, accumulate);
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2, b_desc + 2, id, sf_col, sf_col + 4, 1u);
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 4, b_desc + 4, id, sf_col, sf_col + 4, 1u);
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 6, b_desc + 6, id, sf_col, sf_col + 4, 1u);
+              accumulate = 1;
+              if constexpr (kPair) tc_commit_pair_addr(empty_base + 8 * s);
+              else tc_commit_addr<1>(empty_base + 8 * s);
+              id += kSfIdStep;
+              if (++s == STAGES) {
+                s = 0;
+                phase ^= 1;
+              }
+            }
           }
-          const uint64_t a_desc = a_desc0 + static_cast<uint64_t>(s * (L::kABytes >> 4));
-          const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s * (L::kBBytes >> 4));
-          const uint32_t id = idesc[kb & 3];
-          // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc, b_desc, id, sf_col, sf_col + 4, kb > 0 ? 1u : 0u);
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2, b_desc + 2, id, sf_col, sf_col + 4, 1u);
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 4, b_desc + 4, id, sf_col, sf_col + 4, 1u);
-          mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 6, b_desc + 6, id, sf_col, sf_col + 4, 1u);
-          if constexpr (kPair) tc_commit_pair(&empty_bar[s]);
-          else tc_commit<1>(&empty_bar[s]);
-          if ((kb & 3) == 3 || kb == num_kb - 1) {
-            if constexpr (kPair) tc_commit_pair(&sf_empty[ring]);
-            else tc_commit<1>(&sf_empty[ring]);
-          }
-          if (++s == STAGES) {
-            s = 0;
-            phase ^= 1;
-          }
+          if (!ok) break;
+          if constexpr (kPair) tc_commit_pair(&sf_empty[ring]);
+          else tc_commit<1>(&sf_empty[ring]);
         }
         if (!ok) break;
         if constexpr (kPair) tc_commit_pair(&tmem_full[acc]);
