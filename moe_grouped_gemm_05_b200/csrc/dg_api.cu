@@ -166,17 +166,18 @@ static thread_local int t_force_ctas = 0;
 
 // Heuristic.  Each configuration has a sustained rate measured on B200 with
 // full waves and cold L2 (dense 4096x7168x2048, 8192^3, contiguous and
-// masked workloads, FP8 TFLOP/s): 128-wide tiles run at ~0.62 of the
-// 224/256-wide ones because the per-K-block issue cost of the MMA thread,
-// not the tensor pipe, bounds narrow tiles.  The estimated time of a
-// configuration is its padded work (whole tiles, whole waves of
+// masked workloads, FP8 TFLOP/s).  128-wide tiles run at ~0.65 of the
+// 224-wide ones because the MMA-issuing thread, not the tensor pipe, bounds
+// narrow tiles; 256-wide tiles have a single TMEM accumulator, so their
+// epilogue does not overlap the next tile; 2-CTA tiles add cross-CTA
+// synchronisation without relieving the issuing thread.  The estimated time
+// of a configuration is its padded work (whole tiles, whole waves of
 // co-resident units) divided by that rate.  The masked layout keeps 1-CTA
-// tiles: a 256-row tile wastes half its work on experts with <= 128 valid
-// rows.
+// tiles: a 256-row tile wastes half its work on experts with <= 128 rows.
 static double config_rate(const Config& c) {
-  if (c.bn <= 128) return c.ctas == 2 ? 1270.0 : 1290.0;
-  if (c.bn <= 224) return c.ctas == 2 ? 2100.0 : 2050.0;
-  return c.ctas == 2 ? 2150.0 : 2100.0;
+  if (c.bn <= 128) return c.ctas == 2 ? 1400.0 : 1600.0;
+  if (c.bn <= 224) return c.ctas == 2 ? 2250.0 : 2450.0;
+  return c.ctas == 2 ? 2200.0 : 2250.0;
 }
 
 template <int MODE>
