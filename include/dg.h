@@ -117,6 +117,21 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const voi
  */
 int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb, void* stream);
 
+/*
+ * Per-token FP8 quantisation of activations, fused with the scale packing:
+ * the step before the GEMM that DeepGEMM leaves to its caller (ssnai.com
+ * analysis, "库不做预处理" / "上层完成转置与 FP8/FP4 casting").
+ *   x       : [batch][M][K] activations, BF16 (x_dtype 0) or FP32 (x_dtype 1), finite
+ *   q       : E4M3 [batch][M][K] (written)
+ *   sf      : int32 [batch][ceil(K/512)][align4(M)] packed UE8M0 scales (written,
+ *             padding included): the `sfa` layout of the GEMM entry points.
+ * For every row and 128-wide K group the scale is the smallest power of two s
+ * with max|x|/s <= 448 (1 for an all-zero group, clamped to [2^-127, 2^127])
+ * and q = E4M3(x/s), round to nearest even, saturating.  K % 128 == 0.
+ */
+int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int batch, int M, int K,
+                          void* stream);
+
 /* M alignment of expert segments in the contiguous layout (128). */
 int dg_get_mk_alignment_for_contiguous_layout(void);
 

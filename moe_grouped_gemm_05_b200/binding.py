@@ -46,6 +46,7 @@ def load() -> ctypes.CDLL:
     lib.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
     lib.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
     lib.dg_pack_sf_ue8m0.argtypes = [vp, i32p, i, i, i, vp]
+    lib.dg_quantize_fp8_1x128.argtypes = [vp, i, vp, i32p, i, i, i, vp]
     lib.dg_packed_sf_words.argtypes = [i, i]
     lib.dg_packed_sf_words.restype = ctypes.c_int64
     lib.dg_get_mk_alignment_for_contiguous_layout.argtypes = []
@@ -56,7 +57,8 @@ def load() -> ctypes.CDLL:
     lib.dg_describe_config.argtypes = [i, i, i, i, i, ctypes.c_char_p, i]
     lib.dg_get_last_error.restype = ctypes.c_char_p
     for name in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous", "dg_m_grouped_fp8_gemm_nt_masked",
-                 "dg_pack_sf_ue8m0", "dg_get_device_error", "dg_set_config", "dg_describe_config"):
+                 "dg_pack_sf_ue8m0", "dg_get_device_error", "dg_set_config", "dg_describe_config",
+                 "dg_quantize_fp8_1x128"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -114,6 +116,32 @@ def pack_sf_ue8m0(sf: torch.Tensor) -> torch.Tensor:
     out = torch.empty((batch, kp, mn4), dtype=torch.int32, device=sf.device)
     _check(load().dg_pack_sf_ue8m0(_ptr(s3), _ptr(out), batch, mn, kb, _stream()))
     return out[0] if squeeze else out
+
+
+def quantize_fp8_1x128(x: torch.Tensor, q=None, sf=None):
+    """Per-token 1x128 FP8 quantisation of x[..., M, K] (bf16 or fp32).
+
+    Returns (q float8_e4m3fn [..., M, K], sf int32 [..., ceil(K/512), align4(M)]),
+    the `a` / `sfa` operands of the GEMM entry points.
+    """
+    if x.dtype not in (torch.bfloat16, torch.float32) or not x.is_cuda or not x.is_contiguous():
+        raise TypeError("x must be a contiguous bf16 or fp32 CUDA tensor")
+    if x.dim() < 2:
+        raise ValueError("x must be [..., M, K]")
+    *lead, M, K = x.shape
+    batch = 1
+    for n in lead:
+        batch *= n
+    kp, mn4 = packed_sf_words(M, K // 128)
+    if q is None:
+        q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
+    if sf is None:
+        sf = torch.empty((*lead, kp, mn4), dtype=torch.int32, device=x.device)
+    if tuple(q.shape) != tuple(x.shape) or tuple(sf.shape) != (*lead, kp, mn4):
+        raise ValueError("q / sf shapes do not match x")
+    _check(load().dg_quantize_fp8_1x128(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, _ptr(q), _ptr(sf), batch,
+                                        M, K, _stream()))
+    return q, sf
 
 
 def fp8_gemm_nt(a, sfa, b, sfb, d=None) -> torch.Tensor:

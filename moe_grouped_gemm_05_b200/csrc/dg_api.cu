@@ -13,6 +13,7 @@
 
 #include "dg.h"
 #include "fp8_gemm_kernel.cuh"
+#include "quant_kernel.cuh"
 
 namespace dg {
 
@@ -513,6 +514,35 @@ int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb
   const long long blocks = std::min<long long>((total + threads - 1) / threads, 8LL * di.sms);
   pack_sf_ue8m0_kernel<<<static_cast<int>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
       sf, reinterpret_cast<uint32_t*>(packed), batch, mn, kb, kp, mn4);
+  DG_CUDA_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int batch, int M, int K,
+                          void* stream) {
+  if (!x || !q || !sf) return fail(DG_ERR_NULL, "x, q and sf must be non-NULL");
+  if (x_dtype != 0 && x_dtype != 1) return fail(DG_ERR_UNSUPPORTED, "x_dtype=%d (0: bf16, 1: fp32)", x_dtype);
+  if (!aligned16(x) || !aligned16(q) || !aligned16(sf)) return fail(DG_ERR_ALIGN, "x, q and sf must be 16-byte aligned");
+  if (K <= 0 || K % 128 != 0) return fail(DG_ERR_SHAPE, "K=%d must be a positive multiple of 128", K);
+  if (M < 0 || batch < 0) return fail(DG_ERR_SHAPE, "negative size");
+  const int kp = (K / 128 + 3) / 4;
+  const int mn4 = (M + 3) / 4 * 4;
+  const long long units = static_cast<long long>(batch) * mn4 * kp;
+  if (units == 0) return DG_OK;
+  DeviceInfo di;
+  int r = device_info(&di);
+  if (r) return r;
+  const int threads = 256;
+  const long long blocks = std::min<long long>((units + 7) / 8, 32LL * di.sms);
+  auto st = static_cast<cudaStream_t>(stream);
+  if (x_dtype == 0)
+    quantize_1x128_kernel<__nv_bfloat16><<<static_cast<int>(blocks), threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(q), reinterpret_cast<uint32_t*>(sf), batch, M,
+        K, kp, mn4);
+  else
+    quantize_1x128_kernel<float><<<static_cast<int>(blocks), threads, 0, st>>>(
+        static_cast<const float*>(x), static_cast<uint8_t*>(q), reinterpret_cast<uint32_t*>(sf), batch, M, K, kp,
+        mn4);
   DG_CUDA_TRY(cudaGetLastError());
   return DG_OK;
 }

@@ -222,3 +222,67 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa_words, b, sfb_words, masked_m, d_bits, G
         d_bits[g, :mg] = fp8_gemm_nt(a[g], sfa_words[g], b[g], sfb_words[g], M_max, N, K,
                                      rows=np.arange(mg))
     return bad
+
+
+# ---------------------------------------------------------------------------
+# Per-token 1x128 quantisation (the activation side of the recipe)
+
+
+def e4m3_encode_rne(y: np.ndarray) -> np.ndarray:
+    """E4M3FN codes of float64 values: round to nearest, ties to even, saturating at +-448.
+
+    Negative inputs keep the sign bit even when they round to zero (-0 is 0x80).
+
+    Normal values 2^-6 <= |y| have 3 mantissa bits, so their quantum is
+    2^(floor(log2|y|) - 3); below 2^-6 the quantum is the subnormal step 2^-9.
+    y is divided by its quantum (exact: a power of two), rounded half-to-even,
+    scaled back and clamped to 448; the code is then built field by field.
+    """
+    y = np.asarray(y, dtype=np.float64)
+    a = np.abs(y)
+    _, ex = np.frexp(np.where(a > 0, a, 1.0))
+    lg = ex - 1
+    qexp = np.where(lg < -6, -9, lg - 3)
+    v = np.ldexp(np.rint(np.ldexp(a, -qexp)), qexp)
+    v = np.minimum(v, 448.0)
+    # encode v (a representable magnitude) into exponent / mantissa fields
+    _, ev = np.frexp(np.where(v > 0, v, 1.0))
+    lv = ev - 1
+    sub = v < 2.0 ** -6
+    e_field = np.where(sub, 0, lv + 7)
+    m_field = np.where(sub, np.rint(v / 2.0 ** -9), np.rint((v / np.ldexp(1.0, lv) - 1.0) * 8))
+    code = (e_field.astype(np.int64) << 3) | m_field.astype(np.int64)
+    code = np.where(v == 0, 0, code)
+    sign = np.signbit(y).astype(np.int64) << 7  # negative values keep their sign, -0 included
+    return (code | sign).astype(np.uint8)
+
+
+def pow2_scale_for_amax(amax: np.ndarray) -> np.ndarray:
+    """Smallest power of two s with amax / s <= 448, within UE8M0's [2^-127, 2^127]; 1 for amax = 0."""
+    amax = np.asarray(amax, dtype=np.float64)
+    r = amax / 448.0  # only the comparison with powers of two matters: do it exactly below
+    _, e = np.frexp(np.where(amax > 0, r, 1.0))
+    c = e.astype(np.int64)  # r < 2^e; 2^(e-1) <= r
+    exact_half = np.ldexp(448.0, e - 1) >= amax  # 448 * 2^(e-1) >= amax, decided exactly
+    c = np.where(exact_half, e - 1, e)
+    c = np.clip(c, -127, 127)
+    return np.where(amax > 0, np.ldexp(1.0, c), 1.0)
+
+
+def quantize_fp8_1x128(x: np.ndarray):
+    """Quantises x[..., M, K] per row and 128-wide K group.
+
+    Returns (E4M3 codes with x's shape, packed UE8M0 words [..., ceil(K/512), align4(M)]).
+    The scale of a group is the smallest power of two s with max|x|/s <= 448.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    *lead, M, K = x.shape
+    assert K % BLOCK == 0
+    g = x.reshape(*lead, M, K // BLOCK, BLOCK)
+    s = pow2_scale_for_amax(np.abs(g).max(axis=-1))
+    codes = e4m3_encode_rne(g / s[..., None]).reshape(x.shape)
+    sf = s.astype(np.float32)
+    sf3 = sf.reshape(-1, M, K // BLOCK)
+    words, bad = pack_sf_ue8m0(sf3)
+    assert bad == 0
+    return codes, words.reshape(*lead, *words.shape[1:])

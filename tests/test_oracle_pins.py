@@ -355,3 +355,59 @@ def test_zipf_routing_counts():
 def test_masked_counts_range():
     m = synth.uniform_masked_m(7, 1000, 256)
     assert m.min() >= 0 and m.max() <= 256 and 100 < m.mean() < 156
+
+
+# ---------------------------------------------------------------- activation quantisation
+
+
+def test_e4m3_encode_matches_torch_cast():
+    rng = np.random.default_rng(12)
+    y = np.concatenate([rng.standard_normal(50000) * 100, rng.standard_normal(5000) * 1e-3,
+                        rng.uniform(-448, 448, 20000)])
+    # exact midpoints between neighbouring E4M3 values (ties to even)
+    tab = oracle.e4m3_table()
+    pos = np.sort(tab[(np.arange(256) < 0x7F)])
+    mids = (pos[1:] + pos[:-1]) / 2
+    y = np.concatenate([y, mids, -mids, [0.0, -0.0, 448.0, -448.0]])
+    y = np.clip(y.astype(np.float32).astype(np.float64), -448, 448)
+    got = oracle.fp8_gemm.e4m3_encode_rne(y)
+    ref = torch.from_numpy(y.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+    assert oracle.fp8_gemm.e4m3_encode_rne(np.array([1000.0]))[0] == 0x7E  # saturates
+
+
+def test_pow2_scale_is_smallest_fitting_power_of_two():
+    f = oracle.fp8_gemm.pow2_scale_for_amax
+    assert f(np.array([448.0]))[0] == 1.0 and f(np.array([449.0]))[0] == 2.0
+    assert f(np.array([0.0]))[0] == 1.0
+    one75 = np.float32(1.75)
+    nxt = np.nextafter(one75, np.float32(2))
+    assert f(np.array([float(one75)]))[0] == 2.0 ** -8
+    assert f(np.array([float(nxt)]))[0] == 2.0 ** -7
+    rng = np.random.default_rng(13)
+    a = np.abs(rng.standard_normal(10000) * np.exp(rng.uniform(-40, 40, 10000)))
+    s = f(a)
+    assert np.all(a / s <= 448) and np.all(a / (s / 2) > 448)
+    assert f(np.array([1e-45]))[0] == 2.0 ** -127   # clamped to the UE8M0 range
+
+
+def test_quantize_worked_example():
+    x = np.zeros((2, 128))
+    x[0, 0], x[0, 5] = 448.0, -1.0
+    x[1, 0], x[1, 1] = 449.0, 1e-3
+    codes, words = oracle.fp8_gemm.quantize_fp8_1x128(x)
+    assert codes[0, 0] == 0x7E and codes[0, 5] == 0xB8
+    assert codes[1, 0] == 0x76  # 449 / 2 = 224.5 -> 224 (1.75 * 2^7)
+    w = words.view(np.uint32)
+    assert w[0, 0] == 127 and w[0, 1] == 128 and w[0, 2] == 0  # scales 1, 2; padding row
+
+
+def test_quantize_agrees_with_the_generator_recipe():
+    # the generator quantises with PyTorch's own cast; the oracle encodes by hand
+    x = synth.normal(77, 5 * 384).reshape(5, 384)
+    x[2] *= 1e-3
+    x[3, :128] = 0.0
+    q_gen, s_gen = synth.quantize_rows(x)
+    codes, words = oracle.fp8_gemm.quantize_fp8_1x128(x)
+    assert np.array_equal(codes, q_gen)
+    assert np.array_equal(words, oracle.pack_sf_ue8m0(s_gen[None])[0][0])
