@@ -72,6 +72,20 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
                    int M, int N, int K, void* stream);
 
 /*
+ * Dense FP8 GEMM, NT layout, with the recipe and output options of DeepGEMM's
+ * `fp8_gemm_nt(a, b, d, c=None, recipe=...)` (nightvoyager.top report, "解法哲学";
+ * "1d1d / 1d2d" kernels under "关键设计决策"; the juejin.cn article §2.1's
+ * general GEMM C = alpha*A*B + beta*C with alpha = beta = 1):
+ *   sfb_gran_n : 128 -> B scales per 128x128 block (packed MN = ceil(N/128));
+ *                1   -> B scales per row and 128-wide K block, "1D1D" (packed MN = N).
+ *   c          : optional FP32 [M][N] added to the product (NULL: none); needs d_is_fp32.
+ *   d          : BF16 [M][N] (d_is_fp32 = 0) or FP32 [M][N] (d_is_fp32 = 1).
+ * With c == NULL, sfb_gran_n == 128 and d_is_fp32 == 0 this is dg_fp8_gemm_nt.
+ */
+int dg_fp8_gemm_nt_ex(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const float* c,
+                      void* d, int M, int N, int K, int sfb_gran_n, int d_is_fp32, void* stream);
+
+/*
  * M-grouped GEMM, contiguous layout (juejin.cn article §4 "分组 GEMM（连续布局）":
  * the experts' tokens are concatenated along M, each expert segment aligned
  * to the M block; N and K are shared by all experts).

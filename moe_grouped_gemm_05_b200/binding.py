@@ -47,6 +47,7 @@ def load() -> ctypes.CDLL:
     lib.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
     lib.dg_pack_sf_ue8m0.argtypes = [vp, i32p, i, i, i, vp]
     lib.dg_quantize_fp8_1x128.argtypes = [vp, i, vp, i32p, i, i, i, vp]
+    lib.dg_fp8_gemm_nt_ex.argtypes = [vp, i32p, vp, i32p, vp, vp, i, i, i, i, i, vp]
     lib.dg_packed_sf_words.argtypes = [i, i]
     lib.dg_packed_sf_words.restype = ctypes.c_int64
     lib.dg_get_mk_alignment_for_contiguous_layout.argtypes = []
@@ -58,7 +59,7 @@ def load() -> ctypes.CDLL:
     lib.dg_get_last_error.restype = ctypes.c_char_p
     for name in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous", "dg_m_grouped_fp8_gemm_nt_masked",
                  "dg_pack_sf_ue8m0", "dg_get_device_error", "dg_set_config", "dg_describe_config",
-                 "dg_quantize_fp8_1x128"):
+                 "dg_quantize_fp8_1x128", "dg_fp8_gemm_nt_ex"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -158,6 +159,27 @@ def fp8_gemm_nt(a, sfa, b, sfb, d=None) -> torch.Tensor:
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
         raise ValueError("d must be a contiguous bf16 [M, N] tensor")
     _check(load().dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def fp8_gemm_nt_ex(a, sfa, b, sfb, c=None, d=None, recipe_b: int = 128, out_dtype=torch.bfloat16) -> torch.Tensor:
+    """D = A . B^T (+ C).  recipe_b: rows of B per scale (128 = 128x128 blocks, 1 = per-row "1D1D").
+
+    out_dtype bf16 or float32; c (float32 [M, N]) requires a float32 output.
+    """
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb")
+    M, K = a.shape
+    N, Kb_ = b.shape
+    if Kb_ != K:
+        raise ValueError("a and b disagree on K")
+    if tuple(sfb.shape) != packed_sf_words(-(-N // recipe_b), K // 128) or tuple(sfa.shape) != packed_sf_words(M, K // 128):
+        raise ValueError("packed scale shapes do not match the recipe")
+    if c is not None and (c.dtype != torch.float32 or tuple(c.shape) != (M, N) or not c.is_contiguous()):
+        raise ValueError("c must be a contiguous float32 [M, N] tensor")
+    if d is None:
+        d = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    _check(load().dg_fp8_gemm_nt_ex(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c) if c is not None else None,
+                                    _ptr(d), M, N, K, recipe_b, 1 if d.dtype == torch.float32 else 0, _stream()))
     return d
 
 

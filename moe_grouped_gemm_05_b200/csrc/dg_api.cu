@@ -121,7 +121,7 @@ struct Config {
   KernelFn fn = nullptr;
 };
 
-template <int BN, int STAGES, int MODE, int CTAS>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false>
 static Config make_config() {
   Config c;
   c.bn = BN;
@@ -129,16 +129,26 @@ static Config make_config() {
   c.ctas = CTAS;
   c.smem = Layout<BN, STAGES, CTAS>::kSmemBytes;
   c.num_acc = Layout<BN, STAGES, CTAS>::kNumAcc;
-  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS>);
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32>);
   return c;
 }
 
 // Built configurations.  A 2-CTA tile spans 256 rows, which the contiguous
 // layout (128-row expert alignment) cannot guarantee to be one expert, so the
 // contiguous mode uses single-CTA tiles only.
+// Host-side id of the dense kernels with FP32 output (optionally + C).
+constexpr int MODE_DENSE_F32 = 3;
+
 template <int MODE>
 static const Config* config_table(int* count) {
-  if constexpr (MODE == MODE_CONTIG) {
+  if constexpr (MODE == MODE_DENSE_F32) {
+    static const Config table[] = {
+        make_config<128, 6, MODE_DENSE, 1, true>(), make_config<224, 4, MODE_DENSE, 1, true>(),
+        make_config<256, 4, MODE_DENSE, 1, true>(),
+    };
+    *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
+    return table;
+  } else if constexpr (MODE == MODE_CONTIG) {
     static const Config table[] = {
         make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
     };
@@ -191,7 +201,7 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms) {
   double best_cost = 1e300;
   for (int i = 0; i < n; ++i) {
     const Config& c = t[i];
-    if (MODE == MODE_MASKED && c.ctas != 1) continue;
+    if ((MODE == MODE_MASKED || MODE == MODE_DENSE_F32) && c.ctas != 1) continue;
     const long long tile_m = 128LL * c.ctas;
     const long long m_tiles = (rows_est + tile_m - 1) / tile_m;
     const long long n_tiles = (N + c.bn - 1) / c.bn;
@@ -287,7 +297,7 @@ static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const Ge
 //   B : [GB][N][K] bytes        box 128 x BN/CTAS,         128-byte swizzle
 //   D : [GD][rowsD][N] bf16     box 32 x 32,               64-byte swizzle
 static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const void* b, void* d,
-                      int rowsA, int GA, int N, int K, int GB, int rowsD, int GD) {
+                      int rowsA, int GA, int N, int K, int GB, int rowsD, int GD, bool d_f32 = false) {
   int r;
   if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, rowsA, GA, K,
                     static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A")))
@@ -296,9 +306,13 @@ static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const
                     static_cast<uint64_t>(N) * K, 128, cfg->bn / cfg->ctas, CU_TENSOR_MAP_SWIZZLE_128B,
                     "B")))
     return r;
-  if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, rowsD, GD,
-                    static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(rowsD) * N * 2, 32, 32,
-                    CU_TENSOR_MAP_SWIZZLE_64B, "D")))
+  if (d_f32) {  // 16 FP32 columns (64 B) per box row
+    if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, N, rowsD, GD, static_cast<uint64_t>(N) * 4,
+                      static_cast<uint64_t>(rowsD) * N * 4, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B, "D")))
+      return r;
+  } else if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, d, N, rowsD, GD,
+                           static_cast<uint64_t>(N) * 2, static_cast<uint64_t>(rowsD) * N * 2, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B, "D")))
     return r;
   return DG_OK;
 }
@@ -323,7 +337,7 @@ struct MapEntry {
 };
 
 static int build_maps_cached(CUtensorMap* maps, const Config* cfg, const void* a, const void* b, void* d,
-                             int rowsA, int GA, int N, int K, int GB, int rowsD, int GD) {
+                             int rowsA, int GA, int N, int K, int GB, int rowsD, int GD, bool d_f32 = false) {
   constexpr int kSlots = 64;
   static thread_local MapEntry cache[kSlots];
   MapKey key;
@@ -348,7 +362,7 @@ static int build_maps_cached(CUtensorMap* maps, const Config* cfg, const void* a
     std::memcpy(maps, e.maps, sizeof(e.maps));
     return DG_OK;
   }
-  int r = build_maps(maps, cfg, a, b, d, rowsA, GA, N, K, GB, rowsD, GD);
+  int r = build_maps(maps, cfg, a, b, d, rowsA, GA, N, K, GB, rowsD, GD, d_f32);
   if (r) return r;
   e.valid = true;
   e.key = key;
@@ -356,10 +370,12 @@ static int build_maps_cached(CUtensorMap* maps, const Config* cfg, const void* a
   return DG_OK;
 }
 
-static void fill_scale_args(GemmArgs* args, const int32_t* sfa, const int32_t* sfb, int rowsA, int N, int K) {
+static void fill_scale_args(GemmArgs* args, const int32_t* sfa, const int32_t* sfb, int rowsA, int N, int K,
+                            int sfb_gran = 128) {
   args->kp = (K / 128 + 3) / 4;
   args->mn4a = (rowsA + 3) / 4 * 4;
-  args->nb4 = ((N + 127) / 128 + 3) / 4 * 4;
+  args->sfb_gran = sfb_gran;
+  args->nb4 = ((N + sfb_gran - 1) / sfb_gran + 3) / 4 * 4;
   args->sfa = reinterpret_cast<const uint32_t*>(sfa);
   args->sfb = reinterpret_cast<const uint32_t*>(sfb);
 }
@@ -572,6 +588,42 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
   const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
   return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles, cfg), maps, args,
                             static_cast<cudaStream_t>(stream));
+}
+
+int dg_fp8_gemm_nt_ex(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const float* c,
+                      void* d, int M, int N, int K, int sfb_gran_n, int d_is_fp32, void* stream) {
+  int r = check_common(a, sfa, b, sfb, d, N, K);
+  if (r) return r;
+  if (sfb_gran_n != 1 && sfb_gran_n != 128)
+    return fail(DG_ERR_UNSUPPORTED, "sfb_gran_n=%d must be 1 (per-row B scales) or 128 (128x128 blocks)", sfb_gran_n);
+  if (d_is_fp32 != 0 && d_is_fp32 != 1) return fail(DG_ERR_UNSUPPORTED, "d_is_fp32=%d must be 0 or 1", d_is_fp32);
+  if (c && !d_is_fp32) return fail(DG_ERR_UNSUPPORTED, "accumulating into c needs an FP32 d");
+  if (c && !aligned16(c)) return fail(DG_ERR_ALIGN, "c must be 16-byte aligned");
+  if (M < 0) return fail(DG_ERR_SHAPE, "M=%d must be >= 0", M);
+  if (M == 0) return DG_OK;
+  DeviceInfo di;
+  if ((r = device_info(&di))) return r;
+  const Config* cfg = d_is_fp32 ? choose_config<MODE_DENSE_F32>(M, N, K, di.sms) : choose_config<MODE_DENSE>(M, N, K, di.sms);
+  if (!cfg && d_is_fp32) cfg = find_config<MODE_DENSE_F32>(224, 1);  // forced 2-CTA configs have no FP32 form
+  if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
+  CUtensorMap maps[3];
+  if ((r = build_maps_cached(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1, d_is_fp32 != 0))) return r;
+  GemmArgs args = {};
+  args.rows = M;
+  args.N = N;
+  args.K = K;
+  args.G = 1;
+  args.num_m_blocks = (M + 128 * cfg->ctas - 1) / (128 * cfg->ctas);
+  args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
+  args.raster_m = raster_group(args.num_m_blocks);
+  if (d_is_fp32) args.d32 = static_cast<float*>(d);
+  else args.d = static_cast<__nv_bfloat16*>(d);
+  args.c = c;
+  fill_scale_args(&args, sfa, sfb, M, N, K, sfb_gran_n);
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  if (d_is_fp32)
+    return launch<MODE_DENSE_F32>(cfg, grid_size(di.sms, tiles, cfg), maps, args, static_cast<cudaStream_t>(stream));
+  return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles, cfg), maps, args, static_cast<cudaStream_t>(stream));
 }
 
 int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,

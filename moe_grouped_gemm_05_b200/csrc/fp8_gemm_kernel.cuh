@@ -61,12 +61,15 @@ struct GemmArgs {
   int raster_m;       // rasterisation group height in M blocks
   int kp;             // words of packed scales along K: ceil(K/128/4)
   int mn4a;           // words of packed A scales along M: align4(rows)
-  int nb4;            // words of packed B scales along N: align4(ceil(N/128))
+  int nb4;            // words of packed B scales along N: align4(ceil(N / sfb_gran))
+  int sfb_gran;       // rows of B per scale: 128 (128x128 blocks) or 1 (1x128 per row)
   const uint32_t* sfa;
   const uint32_t* sfb;
   const int32_t* m_indices;
   const int32_t* masked_m;
-  __nv_bfloat16* d;
+  __nv_bfloat16* d;   // BF16 output (OUT_F32 == false)
+  float* d32;         // FP32 output (OUT_F32 == true)
+  const float* c;     // optional FP32 addend [rows][N] (OUT_F32 only), nullptr for none
 };
 
 template <int BN, int STAGES, int CTAS>
@@ -178,7 +181,7 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
   return tl;
 }
 
-template <int BN, int STAGES, int MODE, int CTAS>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const int j = 128 * h + 32 * c + lane;
-            const int nb = (n0 + j) >> 7;
+            const int nb = p.sfb_gran == 1 ? n0 + j : (n0 + j) >> 7;
             wb[h][c] = (j < BN && nb < p.nb4) ? __ldg(sfb_row + nb) : 0u;
           }
         uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
@@ -522,6 +525,55 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + 32 * c, r);
         tmem_wait_ld();
+        const size_t row_g = static_cast<size_t>(zd) * p.rows + m_local;
+        if constexpr (OUT_F32) {
+          // FP32 output, optionally plus C: two 16-column halves of 64 B per row
+          if (p.c != nullptr && valid) {
+            const float4* cp = reinterpret_cast<const float4*>(p.c + row_g * p.N + col0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              if (col0 + 4 * i < p.N) {
+                const float4 cv = __ldg(cp + i);
+                r[4 * i] = __float_as_uint(__uint_as_float(r[4 * i]) + cv.x);
+                r[4 * i + 1] = __float_as_uint(__uint_as_float(r[4 * i + 1]) + cv.y);
+                r[4 * i + 2] = __float_as_uint(__uint_as_float(r[4 * i + 2]) + cv.z);
+                r[4 * i + 3] = __float_as_uint(__uint_as_float(r[4 * i + 3]) + cv.w);
+              }
+            }
+          }
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int colh = col0 + 16 * hf;
+            if (colh >= p.N) break;
+            if (all_valid) {
+              uint8_t* buf = reinterpret_cast<uint8_t*>(epi_base) + (store_count & 1) * L::kEpiBuf;
+              ++store_count;
+              if (lane == 0) bulk_wait_group_read<1>();
+              __syncwarp();
+              uint8_t* rowp = buf + lane * 64;
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int chunk = i ^ ((lane >> 1) & 3);  // 64-byte swizzle
+                *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(
+                    r[16 * hf + 4 * i], r[16 * hf + 4 * i + 1], r[16 * hf + 4 * i + 2], r[16 * hf + 4 * i + 3]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tm_d, buf, colh, row0, zd);
+                bulk_commit_group();
+              }
+            } else if (valid) {
+              uint4* dst = reinterpret_cast<uint4*>(p.d32 + row_g * p.N + colh);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                if (colh + 4 * i < p.N)
+                  dst[i] = make_uint4(r[16 * hf + 4 * i], r[16 * hf + 4 * i + 1], r[16 * hf + 4 * i + 2],
+                                      r[16 * hf + 4 * i + 3]);
+            }
+          }
+          continue;
+        }
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -547,7 +599,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             bulk_commit_group();
           }
         } else if (valid) {
-          const size_t row_g = static_cast<size_t>(zd) * p.rows + m_local;
           __nv_bfloat16* dst = p.d + row_g * p.N + col0;
 #pragma unroll
           for (int i = 0; i < 4; ++i)

@@ -286,3 +286,33 @@ def quantize_fp8_1x128(x: np.ndarray):
     words, bad = pack_sf_ue8m0(sf3)
     assert bad == 0
     return codes, words.reshape(*lead, *words.shape[1:])
+
+
+def fp8_gemm_nt_general_f64(a, sfa_words, b, sfb_words, M, N, K, sfb_gran_n=128, c=None, rows=None):
+    """D = A . B^T (+ C) with per-128-K promotion, unrounded float64.
+
+    sfb_gran_n = 128: B carries one scale per 128x128 block ("1D2D", the
+    default recipe); sfb_gran_n = 1: one scale per row of B and 128-wide K
+    block ("1D1D"), packed with MN = N.  c, if given, is an fp32 [M, N]
+    matrix added to the exact product before the output rounding.
+    """
+    Kb = K // BLOCK
+    assert K % BLOCK == 0 and sfb_gran_n in (1, 128)
+    ea = unpack_sf_ue8m0(sfa_words, M, Kb)[0]
+    eb = unpack_sf_ue8m0(sfb_words, -(-N // sfb_gran_n), Kb)[0]
+    rows = np.arange(M) if rows is None else np.asarray(rows)
+    A = _decode(a[rows])
+    B = _decode(b)
+    acc = np.zeros((len(rows), N), dtype=np.float64)
+    cols = np.arange(N) // sfb_gran_n
+    for kb in range(Kb):
+        ks = slice(kb * BLOCK, (kb + 1) * BLOCK)
+        acc += (A[:, ks] @ B[:, ks].T) * ue8m0_value(ea[rows, kb])[:, None] * ue8m0_value(eb[cols, kb])[None, :]
+    if c is not None:
+        acc += np.asarray(c, dtype=np.float32)[rows].astype(np.float64)
+    return acc
+
+
+def f32_bits_from_f64(x: np.ndarray) -> np.ndarray:
+    """Round float64 to float32 (IEEE round to nearest even, as NumPy's cast); uint32 bits."""
+    return np.asarray(x, dtype=np.float64).astype(np.float32).view(np.uint32)

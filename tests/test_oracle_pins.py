@@ -411,3 +411,59 @@ def test_quantize_agrees_with_the_generator_recipe():
     codes, words = oracle.fp8_gemm.quantize_fp8_1x128(x)
     assert np.array_equal(codes, q_gen)
     assert np.array_equal(words, oracle.pack_sf_ue8m0(s_gen[None])[0][0])
+
+
+# ---------------------------------------------------------------- 1D1D recipe, C accumulation
+
+
+def test_1d1d_all_ones_closed_form_and_block_equivalence():
+    M, N, K = 4, 256, 512
+    a = np.full((M, K), 0x38, np.uint8)
+    b = np.full((N, K), 0x38, np.uint8)
+    rng = np.random.default_rng(14)
+    ea = rng.integers(124, 131, size=(M, 4))
+    eb_row = rng.integers(124, 131, size=(N, 4))
+    g = oracle.fp8_gemm.fp8_gemm_nt_general_f64
+    d = g(a, _pack(np.ldexp(1.0, ea - 127)), b, _pack(np.ldexp(1.0, eb_row - 127)), M, N, K, sfb_gran_n=1)
+    for m in range(M):
+        for n in (0, 5, 129, 255):
+            assert d[m, n] == sum(128 * 2.0 ** (ea[m, k] - 127) * 2.0 ** (eb_row[n, k] - 127) for k in range(4))
+    # per-row scales that are constant over 128-row blocks reproduce the block recipe
+    p = synth.dense_problem(8, 384, 256, seed=15)
+    sa = _pack(p.sfa)
+    per_row = np.repeat(p.sfb, 128, axis=0)[: p.N]
+    d_row = g(p.a, sa, p.b, _pack(per_row), p.M, p.N, p.K, sfb_gran_n=1)
+    d_blk = g(p.a, sa, p.b, _pack(p.sfb), p.M, p.N, p.K, sfb_gran_n=128)
+    assert np.array_equal(d_row, d_blk)
+
+
+def test_1d1d_brute_force_fraction():
+    rng = np.random.default_rng(16)
+    M, N, K = 2, 40, 256
+    finite = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], np.uint8)
+    a = rng.choice(finite, size=(M, K)).astype(np.uint8)
+    b = rng.choice(finite, size=(N, K)).astype(np.uint8)
+    ea = rng.integers(120, 134, size=(M, 2))
+    eb = rng.integers(120, 134, size=(N, 2))
+    d = oracle.fp8_gemm.fp8_gemm_nt_general_f64(a, _pack(np.ldexp(1.0, ea - 127)), b, _pack(np.ldexp(1.0, eb - 127)),
+                                                 M, N, K, sfb_gran_n=1)
+    av, bv = _torch_e4m3(a), _torch_e4m3(b)
+    for m in range(M):
+        for n in range(0, N, 7):
+            tot = Fraction(0)
+            for kb in range(2):
+                s = sum(Fraction(float(av[m, k])) * Fraction(float(bv[n, k])) for k in range(kb * 128, kb * 128 + 128))
+                tot += s * Fraction(2) ** int(ea[m, kb] - 127) * Fraction(2) ** int(eb[n, kb] - 127)
+            assert Fraction(d[m, n]) == tot  # every term is exact in float64 here
+
+
+def test_c_accumulation_adds_exactly():
+    p = synth.dense_problem(8, 128, 256, seed=17)
+    sa, sb = _pack(p.sfa), _pack(p.sfb)
+    c = synth.normal(18, p.M * p.N).reshape(p.M, p.N)
+    g = oracle.fp8_gemm.fp8_gemm_nt_general_f64
+    d0 = g(p.a, sa, p.b, sb, p.M, p.N, p.K)
+    d1 = g(p.a, sa, p.b, sb, p.M, p.N, p.K, c=c)
+    assert np.allclose(d1 - d0, c.astype(np.float64), rtol=0, atol=1e-9 * np.abs(d0).max())
+    assert np.array_equal(oracle.fp8_gemm.f32_bits_from_f64(np.array([1 + 2.0 ** -24, 1 + 3 * 2.0 ** -24])),
+                          np.array([0x3F800000, 0x3F800002], np.uint32))  # ties to even
