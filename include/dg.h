@@ -146,6 +146,37 @@ int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb
 int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int batch, int M, int K,
                           void* stream);
 
+/*
+ * MoE permutation into the contiguous layout ("group_by_expert", the step
+ * before the grouped GEMM in the charles2530.github.io source guide §七) and
+ * the weighted combine after it.
+ *
+ * dg_moe_permute_capacity: rows that always suffice for M_cap,
+ *   align128(T*topk + 127*num_experts).
+ * dg_moe_permute:
+ *   topk_ids : int32 [T][topk], expert of each routed slot, -1 = not routed
+ *   q, sfa   : the tokens' E4M3 codes [T][K] and packed scales [ceil(K/512)][align4(T)]
+ *              (as written by dg_quantize_fp8_1x128)
+ *   a_perm   : E4M3 [M_cap][K]   sfa_perm : int32 [ceil(K/512)][M_cap]
+ *   m_indices: int32 [M_cap]     src_of   : int32 [M_cap] source token of each row (-1: padding)
+ *   row_of   : int32 [T][topk], row of each routed slot (-1: not routed)
+ * Expert segments follow in expert order, each padded with -1 rows to a multiple
+ * of 128; inside a segment slots keep their (token, slot) order, so the result is
+ * deterministic.  Rows past the last segment are -1.  a_perm / sfa_perm / m_indices
+ * feed dg_m_grouped_fp8_gemm_nt_contiguous with M_total = M_cap directly.
+ * Ids outside [-1, num_experts) set DG_DEVERR_BAD_EXPERT and are not routed.
+ * num_experts <= 1024; M_cap >= dg_moe_permute_capacity(...) and a multiple of 128.
+ * dg_moe_unpermute_combine:
+ *   out[t] = bf16_rne( sum_s weights[t][s] * d_perm[row_of[t][s]] ) in FP32 over routed
+ *   slots (weights NULL = 1); d_perm BF16 [>= rows][N], out BF16 [T][N], N % 16 == 0.
+ */
+int dg_moe_permute_capacity(int T, int topk, int num_experts);
+int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, const void* q, const int32_t* sfa, int K,
+                   void* a_perm, int32_t* sfa_perm, int32_t* m_indices, int32_t* row_of, int32_t* src_of, int M_cap,
+                   void* stream);
+int dg_moe_unpermute_combine(const void* d_perm, const int32_t* row_of, const float* weights, int T, int topk, int N,
+                             void* out, void* stream);
+
 /* M alignment of expert segments in the contiguous layout (128). */
 int dg_get_mk_alignment_for_contiguous_layout(void);
 

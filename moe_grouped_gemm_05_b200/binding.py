@@ -48,6 +48,9 @@ def load() -> ctypes.CDLL:
     lib.dg_pack_sf_ue8m0.argtypes = [vp, i32p, i, i, i, vp]
     lib.dg_quantize_fp8_1x128.argtypes = [vp, i, vp, i32p, i, i, i, vp]
     lib.dg_fp8_gemm_nt_ex.argtypes = [vp, i32p, vp, i32p, vp, vp, i, i, i, i, i, vp]
+    lib.dg_moe_permute_capacity.argtypes = [i, i, i]
+    lib.dg_moe_permute.argtypes = [i32p, i, i, i, vp, i32p, i, vp, i32p, i32p, i32p, i32p, i, vp]
+    lib.dg_moe_unpermute_combine.argtypes = [vp, i32p, vp, i, i, i, vp, vp]
     lib.dg_packed_sf_words.argtypes = [i, i]
     lib.dg_packed_sf_words.restype = ctypes.c_int64
     lib.dg_get_mk_alignment_for_contiguous_layout.argtypes = []
@@ -59,7 +62,8 @@ def load() -> ctypes.CDLL:
     lib.dg_get_last_error.restype = ctypes.c_char_p
     for name in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous", "dg_m_grouped_fp8_gemm_nt_masked",
                  "dg_pack_sf_ue8m0", "dg_get_device_error", "dg_set_config", "dg_describe_config",
-                 "dg_quantize_fp8_1x128", "dg_fp8_gemm_nt_ex"):
+                 "dg_quantize_fp8_1x128", "dg_fp8_gemm_nt_ex", "dg_moe_permute_capacity", "dg_moe_permute",
+                 "dg_moe_unpermute_combine"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -213,6 +217,49 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m, d=None) -> torch.Tens
     _check(load().dg_m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d),
                                                    _ptr(masked_m), G, M_max, N, K, _stream()))
     return d
+
+
+def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: torch.Tensor):
+    """Contiguous-layout permutation of routed tokens.
+
+    Returns a dict with a (float8 [M_cap, K]), sfa (int32 [kp, M_cap]), m_indices, src_of ([M_cap]) and
+    row_of ([T, topk]); a / sfa / m_indices are the operands of m_grouped_fp8_gemm_nt_contiguous.
+    """
+    _i32(topk_ids, "topk_ids"), _fp8(q, "q"), _i32(sfa, "sfa")
+    T, topk = topk_ids.shape
+    K = q.shape[1]
+    cap = load().dg_moe_permute_capacity(T, topk, num_experts)
+    if cap < 0:
+        _check(cap)
+    kp = (K // 128 + 3) // 4
+    dev = q.device
+    out = {
+        "a": torch.empty((cap, K), dtype=torch.float8_e4m3fn, device=dev),
+        "sfa": torch.empty((kp, cap), dtype=torch.int32, device=dev),
+        "m_indices": torch.empty((cap,), dtype=torch.int32, device=dev),
+        "src_of": torch.empty((cap,), dtype=torch.int32, device=dev),
+        "row_of": torch.empty((T, topk), dtype=torch.int32, device=dev),
+    }
+    _check(load().dg_moe_permute(_ptr(topk_ids), T, topk, num_experts, _ptr(q), _ptr(sfa), K, _ptr(out["a"]),
+                                 _ptr(out["sfa"]), _ptr(out["m_indices"]), _ptr(out["row_of"]), _ptr(out["src_of"]),
+                                 cap, _stream()))
+    return out
+
+
+def moe_unpermute_combine(d_perm: torch.Tensor, row_of: torch.Tensor, weights=None, out=None) -> torch.Tensor:
+    """out[t] = sum_s weights[t, s] * d_perm[row_of[t, s]] (bf16, FP32 sums)."""
+    if d_perm.dtype != torch.bfloat16 or not d_perm.is_contiguous():
+        raise TypeError("d_perm must be contiguous bf16")
+    _i32(row_of, "row_of")
+    T, topk = row_of.shape
+    N = d_perm.shape[1]
+    if weights is not None and (weights.dtype != torch.float32 or tuple(weights.shape) != (T, topk)):
+        raise ValueError("weights must be float32 [T, topk]")
+    if out is None:
+        out = torch.empty((T, N), dtype=torch.bfloat16, device=d_perm.device)
+    _check(load().dg_moe_unpermute_combine(_ptr(d_perm), _ptr(row_of), _ptr(weights) if weights is not None else None,
+                                           T, topk, N, _ptr(out), _stream()))
+    return out
 
 
 def get_device_error() -> int:

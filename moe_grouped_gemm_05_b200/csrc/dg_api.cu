@@ -14,6 +14,7 @@
 #include "dg.h"
 #include "fp8_gemm_kernel.cuh"
 #include "quant_kernel.cuh"
+#include "moe_kernels.cuh"
 
 namespace dg {
 
@@ -559,6 +560,64 @@ int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int 
     quantize_1x128_kernel<float><<<static_cast<int>(blocks), threads, 0, st>>>(
         static_cast<const float*>(x), static_cast<uint8_t*>(q), reinterpret_cast<uint32_t*>(sf), batch, M, K, kp,
         mn4);
+  DG_CUDA_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+int dg_moe_permute_capacity(int T, int topk, int num_experts) {
+  if (T < 0 || topk <= 0 || num_experts <= 0) return fail(DG_ERR_SHAPE, "bad sizes");
+  const long long rows = static_cast<long long>(T) * topk + 127LL * num_experts;
+  const long long cap = (rows + 127) / 128 * 128;
+  if (cap > 0x7FFFFFFFLL) return fail(DG_ERR_SHAPE, "capacity overflows int");
+  return static_cast<int>(cap);
+}
+
+int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, const void* q, const int32_t* sfa, int K,
+                   void* a_perm, int32_t* sfa_perm, int32_t* m_indices, int32_t* row_of, int32_t* src_of, int M_cap,
+                   void* stream) {
+  if (!topk_ids || !q || !sfa || !a_perm || !sfa_perm || !m_indices || !row_of || !src_of)
+    return fail(DG_ERR_NULL, "every pointer must be non-NULL");
+  if (!aligned16(q) || !aligned16(a_perm) || !aligned16(sfa) || !aligned16(sfa_perm))
+    return fail(DG_ERR_ALIGN, "q, sfa, a_perm and sfa_perm must be 16-byte aligned");
+  if (T < 0 || topk <= 0 || num_experts <= 0 || num_experts > kMoeMaxExperts)
+    return fail(DG_ERR_SHAPE, "T=%d topk=%d num_experts=%d (at most %d experts)", T, topk, num_experts, kMoeMaxExperts);
+  if (K <= 0 || K % 128 != 0) return fail(DG_ERR_SHAPE, "K=%d must be a positive multiple of 128", K);
+  const int cap = dg_moe_permute_capacity(T, topk, num_experts);
+  if (cap < 0) return cap;
+  if (M_cap < cap || M_cap % 128 != 0)
+    return fail(DG_ERR_SHAPE, "M_cap=%d must be a multiple of 128 and >= %d (dg_moe_permute_capacity)", M_cap, cap);
+  const long long n = static_cast<long long>(T) * topk;
+  if (n > 0x7FFFFFFFLL) return fail(DG_ERR_SHAPE, "too many routed slots");
+  DeviceInfo di;
+  int r = device_info(&di);
+  if (r) return r;
+  auto st = static_cast<cudaStream_t>(stream);
+  moe_route_kernel<<<num_experts, kMoeThreads, 0, st>>>(topk_ids, static_cast<int>(n), topk, num_experts, M_cap,
+                                                        m_indices, row_of, src_of);
+  DG_CUDA_TRY(cudaGetLastError());
+  const int kp = (K / 128 + 3) / 4;
+  const long long work = static_cast<long long>(M_cap) * (K / 16);
+  const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 16LL * di.sms));
+  moe_gather_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
+      static_cast<const uint8_t*>(q), reinterpret_cast<const uint32_t*>(sfa), T, K, kp, src_of, M_cap,
+      static_cast<uint8_t*>(a_perm), reinterpret_cast<uint32_t*>(sfa_perm));
+  DG_CUDA_TRY(cudaGetLastError());
+  return DG_OK;
+}
+
+int dg_moe_unpermute_combine(const void* d_perm, const int32_t* row_of, const float* weights, int T, int topk, int N,
+                             void* out, void* stream) {
+  if (!d_perm || !row_of || !out) return fail(DG_ERR_NULL, "d_perm, row_of and out must be non-NULL");
+  if (!aligned16(d_perm) || !aligned16(out)) return fail(DG_ERR_ALIGN, "d_perm and out must be 16-byte aligned");
+  if (T < 0 || topk <= 0 || N <= 0 || N % 16 != 0) return fail(DG_ERR_SHAPE, "T=%d topk=%d N=%d", T, topk, N);
+  const long long work = static_cast<long long>(T) * (N / 8);
+  if (work == 0) return DG_OK;
+  DeviceInfo di;
+  int r = device_info(&di);
+  if (r) return r;
+  const long long blocks = std::min<long long>((work + 255) / 256, 16LL * di.sms);
+  moe_combine_kernel<<<static_cast<int>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(d_perm), row_of, weights, T, topk, N, static_cast<__nv_bfloat16*>(out));
   DG_CUDA_TRY(cudaGetLastError());
   return DG_OK;
 }

@@ -572,8 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       r[16 * hf + 4 * i + 3]);
             }
           }
-          continue;
-        }
+        } else {
         uint32_t packed[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -606,6 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               *reinterpret_cast<uint4*>(dst + 8 * i) =
                   make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
+        }  // BF16 output
       }
       tc_fence_before();
       __syncwarp();

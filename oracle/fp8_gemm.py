@@ -316,3 +316,53 @@ def fp8_gemm_nt_general_f64(a, sfa_words, b, sfb_words, M, N, K, sfb_gran_n=128,
 def f32_bits_from_f64(x: np.ndarray) -> np.ndarray:
     """Round float64 to float32 (IEEE round to nearest even, as NumPy's cast); uint32 bits."""
     return np.asarray(x, dtype=np.float64).astype(np.float32).view(np.uint32)
+
+
+# ---------------------------------------------------------------------------
+# MoE permutation into the contiguous layout, and the weighted combine
+
+
+def moe_permute(topk_ids: np.ndarray, num_experts: int, align: int = BLOCK):
+    """Contiguous-layout permutation of routed token slots (group_by_expert).
+
+    topk_ids[t, s] is the expert of slot s of token t (-1: not routed).  Expert
+    segments follow in expert order; inside a segment the slots keep their
+    (token, slot) order; each segment is padded with -1 rows to a multiple of
+    `align`.  Returns (m_indices [M_total], row_of [T, topk] with -1 for
+    unrouted slots, src_of [M_total] with the source token of each row or -1,
+    M_total, bad) where bad counts ids outside [-1, num_experts).
+    """
+    ids = np.asarray(topk_ids, dtype=np.int64)
+    T, topk = ids.shape
+    flat = ids.reshape(-1)
+    bad = int(((flat < -1) | (flat >= num_experts)).sum())
+    m_indices, src_of = [], []
+    row_of = np.full(T * topk, -1, dtype=np.int64)
+    row = 0
+    for e in range(num_experts):
+        slots = np.nonzero(flat == e)[0]          # ascending (token, slot) order
+        row_of[slots] = row + np.arange(len(slots))
+        padded = -(-len(slots) // align) * align
+        m_indices += [e] * len(slots) + [-1] * (padded - len(slots))
+        src_of += list(slots // topk) + [-1] * (padded - len(slots))
+        row += padded
+    return (np.array(m_indices, dtype=np.int32), row_of.reshape(T, topk).astype(np.int32),
+            np.array(src_of, dtype=np.int32), row, bad)
+
+
+def moe_permute_capacity(T: int, topk: int, num_experts: int, align: int = BLOCK) -> int:
+    """Rows that always suffice for the contiguous layout: align(T*topk + (align-1)*num_experts)."""
+    return -(-(T * topk + (align - 1) * num_experts) // align) * align
+
+
+def moe_unpermute_combine(d_bits: np.ndarray, row_of: np.ndarray, weights=None) -> np.ndarray:
+    """out[t] = bf16( sum_s w[t,s] * D[row_of[t,s]] ) over routed slots, summed in float64."""
+    D = bf16_bits_to_f64(d_bits)
+    T, topk = row_of.shape
+    w = np.ones((T, topk)) if weights is None else np.asarray(weights, dtype=np.float32).astype(np.float64)
+    out = np.zeros((T, D.shape[1]))
+    for s in range(topk):
+        r = row_of[:, s]
+        ok = r >= 0
+        out[ok] += w[ok, s][:, None] * D[r[ok]]
+    return bf16_bits_from_f64(out)

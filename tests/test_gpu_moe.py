@@ -1,0 +1,95 @@
+"""GPU parity of the MoE permutation (bit exact: deterministic layout, copied
+codes and scale words) and the combine, and the whole chain
+quantise -> permute -> contiguous grouped GEMM -> combine against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from moe_grouped_gemm_05_b200 import binding as dg
+from moe_grouped_gemm_05_b200 import synth
+
+from helpers import bits, check_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    dg.get_device_error()
+
+
+def _routing(T, topk, G, seed, drop=0.1):
+    rng = np.random.default_rng(seed)
+    ids = np.stack([rng.permutation(G)[:topk] for _ in range(T)]).astype(np.int32)
+    ids[rng.random((T, topk)) < drop] = -1
+    return ids
+
+
+@pytest.mark.parametrize("T,topk,G,K", [(300, 2, 6, 512), (1, 1, 3, 128), (2048, 8, 32, 640), (64, 4, 256, 256)])
+def test_permute_bit_exact(T, topk, G, K):
+    ids = _routing(T, topk, G, seed=T + G)
+    x = torch.from_numpy(synth.normal(T, T * K).reshape(T, K)).to(torch.bfloat16).cuda()
+    q, sfa = dg.quantize_fp8_1x128(x)
+    out = dg.moe_permute(torch.from_numpy(ids).cuda(), G, q, sfa)
+    torch.cuda.synchronize()
+    assert dg.get_device_error() == 0
+    m, row_of, src, Mt, bad = oracle.fp8_gemm.moe_permute(ids, G)
+    cap = out["m_indices"].shape[0]
+    assert cap == oracle.fp8_gemm.moe_permute_capacity(T, topk, G)
+    gm = out["m_indices"].cpu().numpy()
+    gs = out["src_of"].cpu().numpy()
+    assert np.array_equal(gm[:Mt], m) and (gm[Mt:] == -1).all()
+    assert np.array_equal(gs[:Mt], src) and (gs[Mt:] == -1).all()
+    assert np.array_equal(out["row_of"].cpu().numpy(), row_of)
+    valid = np.nonzero(m >= 0)[0]
+    qn = q.view(torch.uint8).cpu().numpy()
+    an = out["a"].view(torch.uint8).cpu().numpy()
+    assert np.array_equal(an[valid], qn[src[valid]])
+    sf_src = sfa.cpu().numpy()
+    sf_out = out["sfa"].cpu().numpy()
+    assert np.array_equal(sf_out[:, valid], sf_src[:, src[valid]])
+    assert (sf_out[:, gm < 0] == 0).all()
+
+
+def test_permute_flags_bad_ids():
+    ids = np.array([[0, 5], [1, -3]], np.int32)
+    x = torch.ones((2, 128), dtype=torch.bfloat16, device="cuda")
+    q, sfa = dg.quantize_fp8_1x128(x)
+    out = dg.moe_permute(torch.from_numpy(ids).cuda(), 2, q, sfa)
+    assert dg.get_device_error() & dg.DG_DEVERR_BAD_EXPERT
+    assert out["row_of"].cpu().numpy().tolist() == [[0, -1], [128, -1]]
+
+
+def test_moe_chain_matches_oracle():
+    T, topk, G, K, N = 700, 2, 5, 1024, 384
+    ids = _routing(T, topk, G, seed=3, drop=0.05)
+    x = torch.from_numpy(synth.normal(5, T * K).reshape(T, K)).to(torch.bfloat16)
+    w = synth.contiguous_problem(G, N, K, rows=0, seed=6, counts=[1] * G)   # expert weights B[G][N][K]
+    sb, _ = oracle.pack_sf_ue8m0(w.sfb)
+    gate = np.random.default_rng(7).random((T, topk)).astype(np.float32)
+    # GPU chain
+    q, sfa = dg.quantize_fp8_1x128(x.cuda())
+    per = dg.moe_permute(torch.from_numpy(ids).cuda(), G, q, sfa)
+    d = dg.m_grouped_fp8_gemm_nt_contiguous(per["a"], per["sfa"], torch.from_numpy(w.b).cuda().view(torch.float8_e4m3fn),
+                                            torch.from_numpy(sb).cuda(), per["m_indices"])
+    out = dg.moe_unpermute_combine(d, per["row_of"], torch.from_numpy(gate).cuda())
+    torch.cuda.synchronize()
+    assert dg.get_device_error() == 0
+    # oracle chain
+    codes, words = oracle.fp8_gemm.quantize_fp8_1x128(x.float().numpy().astype(np.float64))
+    m, row_of, src, Mt, _ = oracle.fp8_gemm.moe_permute(ids, G)
+    rows = np.nonzero(m >= 0)[0]
+    a_perm = np.zeros((Mt, K), np.uint8)
+    a_perm[rows] = codes[src[rows]]
+    sa_src = oracle.unpack_sf_ue8m0(words, T, K // 128)[0]
+    sa_perm = np.ones((Mt, K // 128), np.float32)
+    sa_perm[rows] = np.ldexp(1.0, sa_src[src[rows]].astype(np.int64) - 127)
+    sa_words, _ = oracle.pack_sf_ue8m0(sa_perm[None])
+    d_ref = np.zeros((Mt, N), np.uint16)
+    oracle.m_grouped_fp8_gemm_nt_contiguous(a_perm, sa_words[0], w.b, sb, m, d_ref, G, N, K)
+    check_close(bits(d)[rows], d_ref[rows], "permuted grouped GEMM")
+    ref = oracle.fp8_gemm.moe_unpermute_combine(d_ref, row_of, gate)
+    check_close(bits(out), ref, "combine")

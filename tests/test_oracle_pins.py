@@ -467,3 +467,49 @@ def test_c_accumulation_adds_exactly():
     assert np.allclose(d1 - d0, c.astype(np.float64), rtol=0, atol=1e-9 * np.abs(d0).max())
     assert np.array_equal(oracle.fp8_gemm.f32_bits_from_f64(np.array([1 + 2.0 ** -24, 1 + 3 * 2.0 ** -24])),
                           np.array([0x3F800000, 0x3F800002], np.uint32))  # ties to even
+
+
+# ---------------------------------------------------------------- MoE permute / combine
+
+
+def test_moe_permute_hand_example():
+    ids = np.array([[1, 0], [2, -1], [1, 2], [0, 0]])
+    m, row_of, src, Mt, bad = oracle.fp8_gemm.moe_permute(ids, 3, align=4)
+    assert list(m) == [0, 0, 0, -1, 1, 1, -1, -1, 2, 2, -1, -1]
+    assert row_of.tolist() == [[4, 0], [8, -1], [5, 9], [1, 2]]
+    assert list(src) == [0, 3, 3, -1, 0, 2, -1, -1, 1, 2, -1, -1]
+    assert Mt == 12 and bad == 0
+
+
+def test_moe_permute_invariants():
+    rng = np.random.default_rng(19)
+    T, topk, G = 500, 3, 7
+    ids = rng.integers(-1, G, size=(T, topk))
+    m, row_of, src, Mt, bad = oracle.fp8_gemm.moe_permute(ids, G)
+    assert Mt % 128 == 0 and len(m) == Mt and bad == 0
+    assert Mt <= oracle.fp8_gemm.moe_permute_capacity(T, topk, G)
+    routed = ids >= 0
+    rows = row_of[routed]
+    assert len(set(rows.tolist())) == routed.sum()                 # each routed slot gets its own row
+    assert np.array_equal(m[rows], ids[routed])                    # the row's expert is the slot's
+    assert np.array_equal(src[rows], np.nonzero(routed)[0])        # ... and its source token
+    assert (row_of[~routed] == -1).all() and ((m == -1) == (src == -1)).all()
+    assert (np.diff(m[m >= 0]) >= 0).all()                         # expert segments in order
+    for e in range(G):
+        seg = np.nonzero(m == e)[0]
+        if len(seg):
+            assert seg[0] % 128 == 0 and (np.diff(seg) == 1).all()  # aligned, contiguous
+            assert (np.diff(src[seg]) >= 0).all()                   # stable token order
+
+
+def test_moe_combine_gathers_and_weights():
+    rng = np.random.default_rng(20)
+    D = oracle.bf16_bits_from_f64(rng.integers(-64, 64, size=(16, 32)).astype(np.float64))
+    row_of = np.array([[3, -1], [0, 5], [7, 7]])
+    out = oracle.fp8_gemm.moe_unpermute_combine(D, row_of)
+    Dv = oracle.bf16_bits_to_f64(D)
+    assert np.array_equal(oracle.bf16_bits_to_f64(out[0]), Dv[3])
+    assert np.array_equal(oracle.bf16_bits_to_f64(out[1]), Dv[0] + Dv[5])   # small integers: exact
+    w = np.array([[1.0, 0.0], [0.5, 0.25], [2.0, -1.0]], np.float32)
+    out = oracle.fp8_gemm.moe_unpermute_combine(D, row_of, w)
+    assert np.array_equal(oracle.bf16_bits_to_f64(out[2]), Dv[7])
