@@ -193,11 +193,14 @@ int dg_set_num_sms(int n);
 int dg_get_num_sms(void);
 
 /* Forces the tile configuration of the next calls on this host thread:
- * block_n (a built N tile width) and ctas (1: 128-row tiles on one SM;
- * 2: 256-row tiles on a pair of SMs; 0: whichever is built, 1 first).
- * block_n == 0 restores the heuristic.  The contiguous layout only has
- * 1-CTA tiles.  Returns DG_OK or DG_ERR_UNSUPPORTED. */
-int dg_set_config(int block_n, int ctas);
+ * block_n (a built N tile width), ctas (1: 128-row tiles on one SM;
+ * 2: 256-row tiles on a pair of SMs; 0: whichever is built, 1 first) and
+ * pipes (1: one load/MMA pipeline per CTA; 2: two pipelines taking
+ * alternate tiles, each with its own MMA-issuing thread and accumulator,
+ * 2-CTA 128- and 224-wide tiles only; 0: either, 1 first).  block_n == 0
+ * restores the heuristic.  The contiguous layout only has 1-CTA tiles.
+ * Returns DG_OK or DG_ERR_UNSUPPORTED. */
+int dg_set_config(int block_n, int ctas, int pipes);
 
 /* Describes the configuration the heuristic picks for a problem, as
  * "BMxBNxSTAGES[(2cta)]/grid" in buf (kind: 0 dense, 1 contiguous, 2 masked). */

@@ -57,7 +57,7 @@ def load() -> ctypes.CDLL:
     lib.dg_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.dg_set_num_sms.argtypes = [i]
     lib.dg_get_num_sms.argtypes = []
-    lib.dg_set_config.argtypes = [i, i]
+    lib.dg_set_config.argtypes = [i, i, i]
     lib.dg_describe_config.argtypes = [i, i, i, i, i, ctypes.c_char_p, i]
     lib.dg_get_last_error.restype = ctypes.c_char_p
     for name in ("dg_fp8_gemm_nt", "dg_m_grouped_fp8_gemm_nt_contiguous", "dg_m_grouped_fp8_gemm_nt_masked",
@@ -273,9 +273,9 @@ def set_num_sms(n: int) -> int:
     return load().dg_set_num_sms(n)
 
 
-def set_config(block_n: int, ctas: int = 0) -> None:
-    """Forces the N tile width and 1- or 2-CTA tiles (block_n=0: heuristic)."""
-    _check(load().dg_set_config(block_n, ctas))
+def set_config(block_n: int, ctas: int = 0, pipes: int = 0) -> None:
+    """Forces the N tile width, 1- or 2-CTA tiles and 1 or 2 pipelines per CTA (block_n=0: heuristic)."""
+    _check(load().dg_set_config(block_n, ctas, pipes))
 
 
 def describe_config(kind: str, M: int, N: int, K: int, num_groups: int = 1) -> str:

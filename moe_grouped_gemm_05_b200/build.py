@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libdg.so")
 SOURCES = ["dg_api.cu"]
-DEPS = ["dg_api.cu", "fp8_gemm_kernel.cuh", "ptx.cuh"]
+DEPS = ["dg_api.cu", "fp8_gemm_kernel.cuh", "ptx.cuh", "quant_kernel.cuh", "moe_kernels.cuh"]
 
 
 def nvcc_path() -> str:

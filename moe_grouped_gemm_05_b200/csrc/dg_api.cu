@@ -9,7 +9,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "dg.h"
 #include "fp8_gemm_kernel.cuh"
@@ -119,18 +121,22 @@ struct Config {
   int ctas = 1;
   int smem = 0;
   int num_acc = 1;
+  int pipes = 1;  // load/MMA pipelines per CTA (alternate tiles)
+  int threads = kThreads;
   KernelFn fn = nullptr;
 };
 
-template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1>
 static Config make_config() {
   Config c;
   c.bn = BN;
   c.stages = STAGES;
   c.ctas = CTAS;
-  c.smem = Layout<BN, STAGES, CTAS>::kSmemBytes;
-  c.num_acc = Layout<BN, STAGES, CTAS>::kNumAcc;
-  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32>);
+  c.smem = Layout<BN, STAGES, CTAS, PIPES>::kSmemBytes;
+  c.num_acc = Layout<BN, STAGES, CTAS, PIPES>::kNumAcc;
+  c.pipes = PIPES;
+  c.threads = kThreadsFor<PIPES>;
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES>);
   return c;
 }
 
@@ -159,42 +165,50 @@ static const Config* config_table(int* count) {
     static const Config table[] = {
         make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
         make_config<128, 6, MODE, 2>(), make_config<224, 6, MODE, 2>(), make_config<256, 6, MODE, 2>(),
+        make_config<224, 6, MODE, 2, false, 2>(), make_config<128, 6, MODE, 2, false, 2>(),
     };
     *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
     return table;
   }
 }
 
+// First built configuration with this tile width, CTA count (0: any) and
+// number of pipelines (0: any).
 template <int MODE>
-static const Config* find_config(int bn, int ctas) {
+static const Config* find_config(int bn, int ctas, int pipes = 0) {
   int n = 0;
   const Config* t = config_table<MODE>(&n);
   for (int i = 0; i < n; ++i)
-    if (t[i].bn == bn && (ctas == 0 || t[i].ctas == ctas)) return &t[i];
+    if (t[i].bn == bn && (ctas == 0 || t[i].ctas == ctas) && (pipes == 0 || t[i].pipes == pipes))
+      return &t[i];
   return nullptr;
 }
 
 static thread_local int t_force_ctas = 0;
+static thread_local int t_force_pipes = 0;
 
 // Heuristic.  Each configuration has a sustained rate measured on B200 with
 // full waves and cold L2 (dense 4096x7168x2048, 8192^3, contiguous and
-// masked workloads, FP8 TFLOP/s).  128-wide tiles run at ~0.65 of the
-// 224-wide ones because the MMA-issuing thread, not the tensor pipe, bounds
-// narrow tiles; 256-wide tiles have a single TMEM accumulator, so their
-// epilogue does not overlap the next tile; 2-CTA tiles add cross-CTA
-// synchronisation without relieving the issuing thread.  The estimated time
-// of a configuration is its padded work (whole tiles, whole waves of
-// co-resident units) divided by that rate.  The masked layout keeps 1-CTA
-// tiles: a 256-row tile wastes half its work on experts with <= 128 rows.
+// masked workloads, FP8 TFLOP/s).  Every tcgen05 instruction costs the
+// thread that issues it a fixed ~60-70 cycles, so one issuing thread keeps
+// the tensor pipe only ~65% busy on 224-wide tiles and less on 128-wide
+// ones.  Two pipelines per CTA (two issuing threads, alternate tiles)
+// remove that bound; they pay off with 2-CTA tiles, which also halve the B
+// bytes each SM loads from L2.  The estimated time of a configuration is
+// its padded work (whole tiles, whole waves of co-resident units) divided by
+// that rate.  Problems of at most 128 rows stream B from HBM and run fastest
+// on the configuration with the most CTAs, so they keep 1-CTA tiles; so
+// does the masked layout, where a 256-row tile wastes half its work on
+// experts with <= 128 rows.
 static double config_rate(const Config& c) {
-  if (c.bn <= 128) return c.ctas == 2 ? 1400.0 : 1600.0;
-  if (c.bn <= 224) return c.ctas == 2 ? 2250.0 : 2450.0;
-  return c.ctas == 2 ? 2200.0 : 2250.0;
+  if (c.bn <= 128) return c.ctas == 2 ? (c.pipes == 2 ? 2000.0 : 1400.0) : 1550.0;
+  if (c.bn <= 224) return c.ctas == 2 ? (c.pipes == 2 ? 2700.0 : 2300.0) : 2400.0;
+  return c.ctas == 2 ? 2100.0 : 2250.0;
 }
 
 template <int MODE>
 static const Config* choose_config(long long rows_est, int N, int K, int sms) {
-  if (t_force_bn) return find_config<MODE>(t_force_bn, t_force_ctas);
+  if (t_force_bn) return find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes);
   (void)K;
   int n = 0;
   const Config* t = config_table<MODE>(&n);
@@ -202,7 +216,7 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms) {
   double best_cost = 1e300;
   for (int i = 0; i < n; ++i) {
     const Config& c = t[i];
-    if ((MODE == MODE_MASKED || MODE == MODE_DENSE_F32) && c.ctas != 1) continue;
+    if ((MODE == MODE_MASKED || MODE == MODE_DENSE_F32 || rows_est <= 128) && c.ctas != 1) continue;
     const long long tile_m = 128LL * c.ctas;
     const long long m_tiles = (rows_est + tile_m - 1) / tile_m;
     const long long n_tiles = (N + c.bn - 1) / c.bn;
@@ -227,20 +241,19 @@ static int raster_group(int num_m_blocks) { return std::min(num_m_blocks, 16); }
 // wave.  Queried once per configuration and device.
 static int max_active_pairs(const Config* cfg, int sms) {
   static std::mutex mu;
-  static int cache[64][2][8] = {};
+  static std::map<std::pair<int, const void*>, int> cache;  // (device, kernel) -> pairs
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
-  const int key = (cfg->bn / 32) % 8;
-  const int slot = cfg->stages > 5;
+  if (cudaGetDevice(&dev) != cudaSuccess) return sms / 2;
+  const auto key = std::make_pair(dev, reinterpret_cast<const void*>(cfg->fn));
   std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev][slot][key] == 0) {
+  if (cache.find(key) == cache.end()) {
     if (cudaFuncSetAttribute(reinterpret_cast<const void*>(cfg->fn), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              cfg->smem) != cudaSuccess)
       return sms / 2;
     cudaLaunchConfig_t lc = {};
     cudaLaunchAttribute attr[1];
     lc.gridDim = dim3(sms / 2 * 2);
-    lc.blockDim = dim3(kThreads);
+    lc.blockDim = dim3(cfg->threads);
     lc.dynamicSmemBytes = cfg->smem;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -251,9 +264,9 @@ static int max_active_pairs(const Config* cfg, int sms) {
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, reinterpret_cast<const void*>(cfg->fn), &lc) != cudaSuccess || n <= 0)
       n = sms / 2;
-    cache[dev][slot][key] = std::min(n, sms / 2);
+    cache[key] = std::min(n, sms / 2);
   }
-  return cache[dev][slot][key];
+  return cache[key];
 }
 
 template <int MODE>
@@ -278,7 +291,7 @@ static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const Ge
   cudaLaunchConfig_t lc = {};
   cudaLaunchAttribute attr[1];
   lc.gridDim = dim3(grid);
-  lc.blockDim = dim3(kThreads);
+  lc.blockDim = dim3(cfg->threads);
   lc.dynamicSmemBytes = cfg->smem;
   lc.stream = stream;
   if (cfg->ctas == 2) {
@@ -467,17 +480,20 @@ int dg_get_num_sms(void) {
   return g_num_sms_override > 0 ? std::min(g_num_sms_override, di.sms) : di.sms;
 }
 
-int dg_set_config(int block_n, int ctas) {
+int dg_set_config(int block_n, int ctas, int pipes) {
   if (block_n == 0) {
     t_force_bn = 0;
     t_force_ctas = 0;
+    t_force_pipes = 0;
     return DG_OK;
   }
   if (ctas < 0 || ctas > 2) return fail(DG_ERR_UNSUPPORTED, "ctas=%d must be 0, 1 or 2", ctas);
-  if (!find_config<MODE_DENSE>(block_n, ctas))
-    return fail(DG_ERR_UNSUPPORTED, "block_n=%d with ctas=%d is not built", block_n, ctas);
+  if (pipes < 0 || pipes > 2) return fail(DG_ERR_UNSUPPORTED, "pipes=%d must be 0, 1 or 2", pipes);
+  if (!find_config<MODE_DENSE>(block_n, ctas, pipes))
+    return fail(DG_ERR_UNSUPPORTED, "block_n=%d with ctas=%d, pipes=%d is not built", block_n, ctas, pipes);
   t_force_bn = block_n;
   t_force_ctas = ctas;
+  t_force_pipes = pipes;
   return DG_OK;
 }
 
@@ -499,8 +515,8 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
     if (c) tiles = static_cast<long long>((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   }
   if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
-  snprintf(buf, buflen, "%dx%dx%d%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
-           grid_size(sms, tiles, c));
+  snprintf(buf, buflen, "%dx%dx%d%s%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
+           c->pipes == 2 ? "(2pipe)" : "", grid_size(sms, tiles, c));
   return DG_OK;
 }
 

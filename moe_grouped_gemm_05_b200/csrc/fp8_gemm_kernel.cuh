@@ -24,7 +24,9 @@
 //   warp 1     TMEM owner; in the first CTA of a pair also the MMA issuer:
 //              tcgen05.cp of the scales, tcgen05.mma, commits of stage
 //              releases and finished accumulators (to both CTAs of a pair).
-//   warps 2-5  epilogue: tcgen05.ld of this CTA's accumulator rows, BF16 RNE,
+//   warps 2-5 and the last four warps of the block
+//              epilogue: tcgen05.ld of this CTA's accumulator rows (two warps
+//              per TMEM lane quarter, alternate 32-column chunks), BF16 RNE,
 //              swizzled staging + TMA store for fully valid 32-row slices,
 //              predicated stores for slices holding padding/masked rows.
 //   warp 6     scale producer: for every group of 4 K-blocks, the packed UE8M0
@@ -34,6 +36,17 @@
 //              the words never sits on the TMA issue path.
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of
 // tile i overlaps the MMAs of tile i+1.
+//
+// PIPES = 2 (1-CTA tiles): every tcgen05 instruction costs its issuing thread
+// a fixed ~60-70 cycles, so one thread issuing the 4 MMAs + commit of a
+// 128x224x128 K block spends ~300 of the block's 448 tensor-pipe cycles on
+// issue alone and, with its waits, cannot keep the pipe busy.  The cost is
+// per thread: two threads issuing into two accumulators overlap.  So the CTA
+// runs two copies of the load/issue/scale pipeline (warps 0, 1, 6 and 7, 8,
+// 9), each with half of the stage ring, its own scale ring and scale slots
+// in TMEM, taking alternate tiles of the CTA: tile i goes to pipeline i & 1
+// and accumulator i & 1.  The epilogue warps drain the accumulators in tile
+// order, as with one pipeline.
 #pragma once
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -48,7 +61,11 @@ __device__ int g_dg_error = 0;
 enum : int { MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2 };
 
 constexpr int kBK = 128;
-constexpr int kThreads = 224;
+// warps 0, 1, 6: producer, MMA issuer, scale producer; 2-5 and the last four:
+// epilogue; PIPES = 2 adds a second producer, issuer and scale warp (7, 8, 9)
+template <int PIPES>
+constexpr int kThreadsFor = 32 * (11 + 3 * (PIPES - 1));
+constexpr int kThreads = kThreadsFor<1>;
 constexpr int kMaxMaskedGroups = 512;
 constexpr int kMaxSmem = 232448;                  // opt-in shared memory per block on sm_100
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
@@ -72,9 +89,11 @@ struct GemmArgs {
   const float* c;     // optional FP32 addend [rows][N] (OUT_F32 only), nullptr for none
 };
 
-template <int BN, int STAGES, int CTAS>
+template <int BN, int STAGES, int CTAS, int PIPES = 1>
 struct Layout {
   static_assert(CTAS == 1 || CTAS == 2, "CTAS is 1 or 2");
+  static_assert(PIPES == 1 || (PIPES == 2 && STAGES % 2 == 0), "two pipelines need an even number of stages");
+  static constexpr int kStagesPer = STAGES / PIPES;     // stages of each pipeline's ring
   static_assert(BN % 32 == 0 && (BN / CTAS) % 16 == 0 && BN >= 32 && BN <= 256,
                 "BN must be a multiple of 32 in [32, 256] with BN/CTAS a multiple of 16");
   static constexpr int kTileM = 128 * CTAS;
@@ -88,28 +107,31 @@ struct Layout {
   // BN > 128, 32 rows x 16 B with SFB of columns 128-255 for columns +8..+11.
   static constexpr int kSftMainBytes = 4096;
   static constexpr int kSftBytes = kSftMainBytes + (kNB128 == 2 ? 512 : 0);
-  static constexpr int kEpiBuf = 32 * 32 * 2;           // 32 rows x 32 bf16
-  // TMEM columns: accumulators, then two scale slots of 16 columns (SFA at +0, SFB at +4).
+  static constexpr int kEpiBuf = 32 * 32 * 2;           // 32 rows x 32 bf16 (or x 16 fp32)
+  // TMEM columns: accumulators, then per pipeline two scale slots of 16
+  // columns (SFA at +0, SFB at +4).
   static constexpr int kSfSlotCols = 16;
-  static constexpr int kAccStride = BN <= 128 ? 128 : 256;
-  static constexpr int kNumAcc = (kAccStride + BN + 2 * kSfSlotCols <= 512) ? 2 : 1;
-  static constexpr int kSfBaseCol = (kNumAcc - 1) * kAccStride + ((BN + 15) / 16) * 16;
+  static constexpr int kAccStride = PIPES == 2 ? (BN + 31) / 32 * 32 : (BN <= 128 ? 128 : 256);
+  static constexpr int kNumAcc = (PIPES == 2 || kAccStride + BN + 2 * kSfSlotCols <= 512) ? 2 : 1;
+  static constexpr int kSfBaseCol =
+      PIPES == 2 ? 2 * kAccStride : (kNumAcc - 1) * kAccStride + ((BN + 15) / 16) * 16;
   static constexpr int kTmemCols = 512;
   // shared-memory offsets (from a 1024-byte aligned base)
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSft = kOffB + STAGES * kBBytes;
-  // scale ring depth: 4 groups when shared memory allows, else 2
+  // scale ring depth (per pipeline): 4 groups when shared memory allows, else 2
   static constexpr int kSfRing =
-      (kOffSft + 4 * kSftBytes + 1023) / 1024 * 1024 + 4 * 2 * kEpiBuf + 4096 + (2 * kMaxMaskedGroups + 1) * 4 + 1024 <= kMaxSmem ? 4 : 2;
-  static constexpr int kOffEpi = ((kOffSft + kSfRing * kSftBytes + 1023) / 1024) * 1024;
-  static constexpr int kOffBar = kOffEpi + 4 * 2 * kEpiBuf;
-  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 1 + 2 * 4;
+      (kOffSft + PIPES * 4 * kSftBytes + 1023) / 1024 * 1024 + 8 * kEpiBuf + 4096 +
+                  (2 * kMaxMaskedGroups + 1) * 4 + 1024 <= kMaxSmem ? 4 : 2;
+  static constexpr int kOffEpi = ((kOffSft + PIPES * kSfRing * kSftBytes + 1023) / 1024) * 1024;
+  static constexpr int kOffBar = kOffEpi + 8 * kEpiBuf;  // one staging buffer per epilogue warp
+  static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 2 * PIPES * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag
   static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
   static constexpr int kSmemBytes = kOffGroups + (2 * kMaxMaskedGroups + 1) * 4 + 1024;
   static_assert(kSmemBytes <= kMaxSmem, "shared-memory budget exceeded");
-  static_assert(kSfBaseCol + 2 * kSfSlotCols <= kTmemCols, "TMEM budget exceeded");
+  static_assert(kSfBaseCol + PIPES * 2 * kSfSlotCols <= kTmemCols, "TMEM budget exceeded");
 };
 
 struct Tile {
@@ -181,11 +203,11 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
   return tl;
 }
 
-template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1>
+__global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
-  using L = Layout<BN, STAGES, CTAS>;
+  using L = Layout<BN, STAGES, CTAS, PIPES>;
   constexpr bool kPair = CTAS == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -195,9 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* tmem_full = bars + 2 * STAGES;
   uint64_t* tmem_empty = bars + 2 * STAGES + 2;
-  uint64_t* final_bar = bars + 2 * STAGES + 4;
-  uint64_t* sf_full = bars + 2 * STAGES + 5;
-  uint64_t* sf_empty = sf_full + L::kSfRing;
+  uint64_t* final_bar = bars + 2 * STAGES + 4;  // one per pipeline
+  uint64_t* sf_full = bars + 2 * STAGES + 6;    // [pipeline][ring]
+  uint64_t* sf_empty = sf_full + PIPES * L::kSfRing;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
   int* prefix = reinterpret_cast<int*>(smem + L::kOffGroups);
@@ -209,6 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = kPair ? cluster_cta_rank() : 0;
   const int unit0 = kPair ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
   const int units = kPair ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
+  // pipeline of this warp (warps 7, 8, 9 mirror warps 0, 1, 6) and its share of the rings
+  constexpr int kEpiWarp2 = PIPES == 2 ? 10 : 7;  // first warp of the second epilogue set
+  const int pipe = (PIPES == 2 && warp >= 7 && warp < kEpiWarp2) ? 1 : 0;
+  const int sbase = pipe * L::kStagesPer;
+  const int rbase = pipe * L::kSfRing;
+  // With two pipelines, the i-th tile this CTA computes (skipped tiles not
+  // counted) belongs to pipeline i & 1.
+  auto take = [&](uint32_t& li) { return PIPES == 1 || static_cast<int>(li++ & 1) == pipe; };
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -218,10 +248,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tmem_full[i], 1);
-      mbar_init(&tmem_empty[i], 4 * CTAS);
+      mbar_init(&tmem_empty[i], 8 * CTAS);
+      mbar_init(&final_bar[i], 1);
     }
-    mbar_init(final_bar, 1);
-    for (int i = 0; i < L::kSfRing; ++i) {
+    for (int i = 0; i < PIPES * L::kSfRing; ++i) {
       mbar_init(&sf_full[i], CTAS);
       mbar_init(&sf_empty[i], 1);
     }
@@ -267,11 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int ntiles = total_tiles<MODE>(p, prefix);
 
-  if (warp == 0) {
+  if (warp == 0 || (PIPES == 2 && warp == 7)) {
     // ============================================================ producer
     // Barrier of stage s in the MMA-issuing CTA, as a shared::cluster address.
     const uint32_t full0 = kPair ? mapa_shared(smem_u32(full_bar), 0) : smem_u32(full_bar);
-    uint32_t it = 0;
+    uint32_t it = 0, li = 0;
     bool ok = true;
     for (int t = unit0; t < ntiles && ok; t += units) {
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
@@ -283,11 +313,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (MODE == MODE_MASKED) {
         grp_a = grp_b = tl.g;
       }
+      if (!take(li)) continue;
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
       for (int kb = 0; kb < num_kb; ++kb, ++it) {
-        const int s = it % STAGES;
-        ok = wait_phase<false>(&empty_bar[s], ((it / STAGES) & 1) ^ 1, abort_flag);
+        const int s = sbase + static_cast<int>(it % L::kStagesPer);
+        ok = wait_phase<false>(&empty_bar[s], ((it / L::kStagesPer) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (lane == 0) {
@@ -310,11 +341,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     // Drain: every load this CTA's barriers track must land before the CTA exits.
     if (lane == 0 && (!kPair || rank == 0)) {
-      const uint32_t first = it > static_cast<uint32_t>(STAGES) ? it - STAGES : 0;
-      for (uint32_t i = first; i < it; ++i) wait_phase_drain(&full_bar[i % STAGES], (i / STAGES) & 1);
+      const uint32_t first = it > static_cast<uint32_t>(L::kStagesPer) ? it - L::kStagesPer : 0;
+      for (uint32_t i = first; i < it; ++i)
+        wait_phase_drain(&full_bar[sbase + i % L::kStagesPer], (i / L::kStagesPer) & 1);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 || (PIPES == 2 && warp == 8)) {
     // ============================================================ MMA issuer
     // A single thread issues.  Each tcgen05 instruction costs the issuing
     // thread ~60 cycles and every other instruction a few more, against 448
@@ -324,16 +356,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // are precomputed, stage/phase counters are incremental and barrier polls
     // take an inline fast path.
     if ((!kPair || rank == 0) && lane == 0) {
-      const uint32_t a_lo0 = static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffA), 16, 1024, 2));
-      const uint32_t b_lo0 = static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffB), 16, 1024, 2));
+      const uint32_t a_lo0 =
+          static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffA + sbase * L::kABytes), 16, 1024, 2));
+      const uint32_t b_lo0 =
+          static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffB + sbase * L::kBBytes), 16, 1024, 2));
       const uint32_t desc_hi = static_cast<uint32_t>(make_smem_desc(0, 16, 1024, 2) >> 32);
       const uint32_t idesc0 = make_idesc_mxf8(L::kTileM, BN, 0, 0);
       constexpr uint32_t kSfIdStep = (1u << 4) | (1u << 29);  // +1 in both scale-factor byte selectors
-      const uint32_t full_base = smem_u32(full_bar);
-      const uint32_t empty_base = smem_u32(empty_bar);
-      uint32_t s = 0, phase = 0, local_tile = 0, sf_group = 0;
+      const uint32_t full_base = smem_u32(full_bar + sbase);
+      const uint32_t empty_base = smem_u32(empty_bar + sbase);
+      uint32_t s = 0, phase = 0, own = 0, li = 0, sf_group = 0;
       bool ok = true;
-      const uint32_t sft_lo0 = static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffSft), 128, 256, 0));
+      const uint32_t sft_lo0 = static_cast<uint32_t>(
+          make_smem_desc(smem_u32(smem + L::kOffSft + rbase * L::kSftBytes), 128, 256, 0));
+      const uint32_t sf_slot0 = tmem_base + L::kSfBaseCol + pipe * 2 * L::kSfSlotCols;
       const uint32_t sft_hi = static_cast<uint32_t>(make_smem_desc(0, 128, 256, 0) >> 32);
       const uint32_t sfx_hi = static_cast<uint32_t>(make_smem_desc(0, 0, 128, 0) >> 32);
       for (int t = unit0; t < ntiles && ok; t += units) {
@@ -342,9 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
           if (e < 0 || e >= p.G) continue;
         }
-        const uint32_t acc = L::kNumAcc == 1 ? 0 : (local_tile & 1);
-        const uint32_t acc_use = L::kNumAcc == 1 ? local_tile : (local_tile >> 1);
-        ++local_tile;
+        if (!take(li)) continue;
+        // one pipeline: alternate accumulators; two: accumulator = pipeline
+        const uint32_t acc = PIPES == 2 ? pipe : (L::kNumAcc == 1 ? 0 : (own & 1));
+        const uint32_t acc_use = (PIPES == 2 || L::kNumAcc == 1) ? own : (own >> 1);
+        ++own;
         if (!mbar_try_wait(&tmem_empty[acc], (acc_use & 1) ^ 1))
           ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
         if (!ok) break;
@@ -353,18 +391,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t accumulate = 0;
         for (int kb0 = 0; kb0 < num_kb && ok; kb0 += 4, ++sf_group) {
           const uint32_t ring = sf_group % L::kSfRing;
-          const uint32_t sf_col = tmem_base + L::kSfBaseCol + (sf_group & 1) * L::kSfSlotCols;
+          const uint32_t sf_col = sf_slot0 + (sf_group & 1) * L::kSfSlotCols;
           // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
           if (sf_group >= 2) {
-            uint64_t* b = &sf_empty[(sf_group - 2) % L::kSfRing];
+            uint64_t* b = &sf_empty[rbase + (sf_group - 2) % L::kSfRing];
             const uint32_t par = ((sf_group - 2) / L::kSfRing) & 1;
             if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag);
           }
           // acquire at cluster scope: pairs with the scale producers' release (their
           // shared-memory writes are read by tcgen05.cp)
-          if (ok && !(kPair ? mbar_try_wait_cluster(&sf_full[ring], (sf_group / L::kSfRing) & 1)
-                            : mbar_try_wait(&sf_full[ring], (sf_group / L::kSfRing) & 1)))
-            ok = wait_phase<kPair>(&sf_full[ring], (sf_group / L::kSfRing) & 1, abort_flag);
+          if (ok && !(kPair ? mbar_try_wait_cluster(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1)
+                            : mbar_try_wait(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1)))
+            ok = wait_phase<kPair>(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
           {
@@ -380,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
               if (!mbar_try_wait_addr(full_base + 8 * s, phase)) {
-                ok = wait_phase<false>(&full_bar[s], phase, abort_flag);
+                ok = wait_phase<false>(&full_bar[sbase + s], phase, abort_flag);
                 if (!ok) break;
               }
               const uint64_t a_desc = (static_cast<uint64_t>(desc_hi) << 32) | (a_lo0 + s * (L::kABytes >> 4));
@@ -394,29 +432,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               if constexpr (kPair) tc_commit_pair_addr(empty_base + 8 * s);
               else tc_commit_addr<1>(empty_base + 8 * s);
               id += kSfIdStep;
-              if (++s == STAGES) {
+              if (++s == L::kStagesPer) {
                 s = 0;
                 phase ^= 1;
               }
             }
           }
           if (!ok) break;
-          if constexpr (kPair) tc_commit_pair(&sf_empty[ring]);
-          else tc_commit<1>(&sf_empty[ring]);
+          if constexpr (kPair) tc_commit_pair(&sf_empty[rbase + ring]);
+          else tc_commit<1>(&sf_empty[rbase + ring]);
         }
         if (!ok) break;
         if constexpr (kPair) tc_commit_pair(&tmem_full[acc]);
         else tc_commit<1>(&tmem_full[acc]);
       }
       // Drain: all MMAs / copies issued by this thread complete before TMEM is freed.
-      tc_commit<CTAS>(final_bar);
-      wait_phase_drain(final_bar, 0);
+      tc_commit<CTAS>(&final_bar[pipe]);
+      wait_phase_drain(&final_bar[pipe], 0);
     }
     __syncwarp();
-  } else if (warp == 6) {
+  } else if (warp == 6 || (PIPES == 2 && warp == 9)) {
     // ============================================================ scale producer
-    const uint32_t sf_full0 = kPair ? mapa_shared(smem_u32(sf_full), 0) : smem_u32(sf_full);
-    uint32_t group = 0;
+    const uint32_t sf_full0 = kPair ? mapa_shared(smem_u32(sf_full + rbase), 0) : smem_u32(sf_full + rbase);
+    uint32_t group = 0, li = 0;
     bool ok = true;
     for (int t = unit0; t < ntiles && ok; t += units) {
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
@@ -428,11 +466,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (MODE == MODE_MASKED) {
         grp_a = grp_b = tl.g;
       }
+      if (!take(li)) continue;
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
       for (int kp = 0; kp < p.kp; ++kp, ++group) {
         const uint32_t ring = group % L::kSfRing;
-        ok = wait_phase<false>(&sf_empty[ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag);
+        ok = wait_phase<false>(&sf_empty[rbase + ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         // lane r gathers rows / columns r, r+32, r+64, r+96 of each 128-group
@@ -453,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nb = p.sfb_gran == 1 ? n0 + j : (n0 + j) >> 7;
             wb[h][c] = (j < BN && nb < p.nb4) ? __ldg(sfb_row + nb) : 0u;
           }
-        uint8_t* sft = smem + L::kOffSft + ring * L::kSftBytes;
+        uint8_t* sft = smem + L::kOffSft + (rbase + ring) * L::kSftBytes;
         const uint4 va = make_uint4(wa[0], wa[1], wa[2], wa[3]);
         const uint4 vb = make_uint4(wb[0][0], wb[0][1], wb[0][2], wb[0][3]);
 #pragma unroll
@@ -471,16 +510,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
           // the words are read by the tensor core on behalf of the MMA-issuing CTA
           if constexpr (kPair) mbar_arrive_cluster(sf_full0 + 8 * ring);
-          else mbar_arrive(&sf_full[ring]);
+          else mbar_arrive(&sf_full[rbase + ring]);
         }
       }
     }
   } else {
     // ============================================================ epilogue
+    // Eight warps: two per TMEM lane quarter (q = warp % 4), the first of
+    // each pair taking the even 32-column chunks of the tile, the second the
+    // odd ones.  The tcgen05.ld of a warp's next chunk is in flight while the
+    // current one is converted and stored.
     const int q = warp % 4;  // TMEM lane quarter this warp may access
-    __nv_bfloat16* epi_base = reinterpret_cast<__nv_bfloat16*>(smem + L::kOffEpi + (warp - 2) * 2 * L::kEpiBuf);
+    const int half = warp >= kEpiWarp2 ? 1 : 0;
+    const int epi_idx = half ? 4 + (warp - kEpiWarp2) : warp - 2;
+    uint8_t* buf = smem + L::kOffEpi + epi_idx * L::kEpiBuf;  // staging for one TMA store
     const uint32_t empty0 = kPair ? mapa_shared(smem_u32(tmem_empty), 0) : smem_u32(tmem_empty);
-    uint32_t local_tile = 0, store_count = 0;
+    constexpr int kChunks = BN / 32;
+    constexpr int kMaxMine = (kChunks + 1) / 2;
+    const int nmine = half == 0 ? (kChunks + 1) / 2 : kChunks / 2;
+    uint32_t local_tile = 0;
     for (int t = unit0; t < ntiles; t += units) {
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
       int expert = 0;
@@ -508,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (MODE == MODE_CONTIG) {
         const int idx = __ldg(&p.m_indices[m_local]);
         valid = idx == expert;
-        if (!valid && idx != -1 && tl.n_blk == 0)
+        if (!valid && idx != -1 && tl.n_blk == 0 && half == 0)
           atomicOr(&g_dg_error, (idx >= 0 && idx < p.G) ? 0x8 : 0x2);
       } else {
         valid = m_local < counts[tl.g];
@@ -517,15 +565,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool any_valid = __any_sync(0xffffffffu, valid);
       const int n0 = tl.n_blk * BN;
       const int zd = (MODE == MODE_MASKED) ? tl.g : 0;
+      const size_t row_g = static_cast<size_t>(zd) * p.rows + m_local;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * L::kAccStride;
-#pragma unroll 1
-      for (int c = 0; c < BN / 32 && any_valid; ++c) {
-        const int col0 = n0 + 32 * c;
-        if (col0 >= p.N) break;
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + 32 * c, r);
-        tmem_wait_ld();
-        const size_t row_g = static_cast<size_t>(zd) * p.rows + m_local;
+
+      // Converts and stores one 32-column chunk held in rr (lane = row).
+      auto store_chunk = [&](uint32_t (&rr)[32], int col0) {
         if constexpr (OUT_F32) {
           // FP32 output, optionally plus C: two 16-column halves of 64 B per row
           if (p.c != nullptr && valid) {
@@ -534,10 +578,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 8; ++i) {
               if (col0 + 4 * i < p.N) {
                 const float4 cv = __ldg(cp + i);
-                r[4 * i] = __float_as_uint(__uint_as_float(r[4 * i]) + cv.x);
-                r[4 * i + 1] = __float_as_uint(__uint_as_float(r[4 * i + 1]) + cv.y);
-                r[4 * i + 2] = __float_as_uint(__uint_as_float(r[4 * i + 2]) + cv.z);
-                r[4 * i + 3] = __float_as_uint(__uint_as_float(r[4 * i + 3]) + cv.w);
+                rr[4 * i] = __float_as_uint(__uint_as_float(rr[4 * i]) + cv.x);
+                rr[4 * i + 1] = __float_as_uint(__uint_as_float(rr[4 * i + 1]) + cv.y);
+                rr[4 * i + 2] = __float_as_uint(__uint_as_float(rr[4 * i + 2]) + cv.z);
+                rr[4 * i + 3] = __float_as_uint(__uint_as_float(rr[4 * i + 3]) + cv.w);
               }
             }
           }
@@ -546,16 +590,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int colh = col0 + 16 * hf;
             if (colh >= p.N) break;
             if (all_valid) {
-              uint8_t* buf = reinterpret_cast<uint8_t*>(epi_base) + (store_count & 1) * L::kEpiBuf;
-              ++store_count;
-              if (lane == 0) bulk_wait_group_read<1>();
+              if (lane == 0) bulk_wait_group_read<0>();  // previous store has read the buffer
               __syncwarp();
               uint8_t* rowp = buf + lane * 64;
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
                 const int chunk = i ^ ((lane >> 1) & 3);  // 64-byte swizzle
                 *reinterpret_cast<uint4*>(rowp + chunk * 16) = make_uint4(
-                    r[16 * hf + 4 * i], r[16 * hf + 4 * i + 1], r[16 * hf + 4 * i + 2], r[16 * hf + 4 * i + 3]);
+                    rr[16 * hf + 4 * i], rr[16 * hf + 4 * i + 1], rr[16 * hf + 4 * i + 2], rr[16 * hf + 4 * i + 3]);
               }
               fence_proxy_async_smem();
               __syncwarp();
@@ -568,44 +610,57 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
               for (int i = 0; i < 4; ++i)
                 if (colh + 4 * i < p.N)
-                  dst[i] = make_uint4(r[16 * hf + 4 * i], r[16 * hf + 4 * i + 1], r[16 * hf + 4 * i + 2],
-                                      r[16 * hf + 4 * i + 3]);
+                  dst[i] = make_uint4(rr[16 * hf + 4 * i], rr[16 * hf + 4 * i + 1], rr[16 * hf + 4 * i + 2],
+                                      rr[16 * hf + 4 * i + 3]);
             }
           }
         } else {
-        uint32_t packed[16];
+          uint32_t packed[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-          packed[i] = *reinterpret_cast<uint32_t*>(&h);
-        }
-        if (all_valid) {
-          __nv_bfloat16* buf = epi_base + (store_count & 1) * (L::kEpiBuf / 2);
-          ++store_count;
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
-          uint8_t* rowp = reinterpret_cast<uint8_t*>(buf) + lane * 64;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int chunk = i ^ ((lane >> 1) & 3);  // 64-byte swizzle
-            *reinterpret_cast<uint4*>(rowp + chunk * 16) =
-                make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(rr[2 * i]), __uint_as_float(rr[2 * i + 1]));
+            packed[i] = *reinterpret_cast<uint32_t*>(&h2);
           }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&tm_d, buf, col0, row0, zd);
-            bulk_commit_group();
-          }
-        } else if (valid) {
-          __nv_bfloat16* dst = p.d + row_g * p.N + col0;
+          if (all_valid) {
+            if (lane == 0) bulk_wait_group_read<0>();  // previous store has read the buffer
+            __syncwarp();
+            uint8_t* rowp = buf + lane * 64;
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (col0 + 8 * i < p.N)
-              *reinterpret_cast<uint4*>(dst + 8 * i) =
+            for (int i = 0; i < 4; ++i) {
+              const int chunk = i ^ ((lane >> 1) & 3);  // 64-byte swizzle
+              *reinterpret_cast<uint4*>(rowp + chunk * 16) =
                   make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tm_d, buf, col0, row0, zd);
+              bulk_commit_group();
+            }
+          } else if (valid) {
+            __nv_bfloat16* dst = p.d + row_g * p.N + col0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (col0 + 8 * i < p.N)
+                *reinterpret_cast<uint4*>(dst + 8 * i) =
+                    make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
         }
-        }  // BF16 output
+      };
+
+      if (any_valid) {
+        uint32_t r[2][32];
+        if (nmine > 0 && n0 + 32 * half < p.N) tmem_ld_32x32b_x32(t_row + 32 * half, r[0]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < kMaxMine; ++i) {
+          const int c = half + 2 * i;
+          const int col0 = n0 + 32 * c;
+          if (i >= nmine || col0 >= p.N) break;
+          if (i + 1 < nmine && col0 + 64 < p.N) tmem_ld_32x32b_x32(t_row + 32 * (c + 2), r[(i + 1) & 1]);
+          store_chunk(r[i & 1], col0);
+          tmem_wait_ld();
+        }
       }
       tc_fence_before();
       __syncwarp();

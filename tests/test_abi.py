@@ -76,8 +76,11 @@ def test_pack_argument_errors(lib):
 
 
 def test_config_override(lib):
-    assert lib.dg_set_config(96, 0) == -4
-    assert lib.dg_set_config(128, 3) == -4
-    assert lib.dg_set_config(128, 0) == 0
-    assert lib.dg_set_config(224, 2) == 0
-    assert lib.dg_set_config(0, 0) == 0
+    assert lib.dg_set_config(96, 0, 0) == -4
+    assert lib.dg_set_config(128, 3, 0) == -4
+    assert lib.dg_set_config(256, 0, 2) == -4   # two pipelines: 128- and 224-wide 2-CTA tiles only
+    assert lib.dg_set_config(224, 1, 2) == -4
+    assert lib.dg_set_config(128, 0, 0) == 0
+    assert lib.dg_set_config(224, 2, 0) == 0
+    assert lib.dg_set_config(224, 2, 2) == 0
+    assert lib.dg_set_config(0, 0, 0) == 0

@@ -48,7 +48,7 @@ def _row_scales(N, K, seed):
     return np.ldexp(1.0, rng.integers(-10, 3, size=(N, K // 128))).astype(np.float32)
 
 
-@pytest.mark.parametrize("cfg", [(128, 1), (224, 1), (256, 1), (224, 2)])
+@pytest.mark.parametrize("cfg", [(128, 1), (224, 1), (256, 1), (224, 2), (224, 2, 2)])
 @pytest.mark.parametrize("shape", [(200, 336, 384), (256, 512, 1024)])
 def test_1d1d_bf16(cfg, shape):
     M, N, K = shape

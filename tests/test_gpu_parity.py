@@ -13,7 +13,8 @@ from helpers import bits, check_close, packed, to_device
 
 pytestmark = pytest.mark.gpu
 
-BUILT = [(128, 1), (224, 1), (256, 1), (128, 2), (224, 2), (256, 2)]  # (block_n, ctas)
+# (block_n, ctas, pipes)
+BUILT = [(128, 1, 1), (224, 1, 1), (256, 1, 1), (128, 2, 1), (224, 2, 1), (256, 2, 1), (224, 2, 2), (128, 2, 2)]
 BUILT_1CTA = [c for c in BUILT if c[1] == 1]
 SENTINEL = 0xDEAD
 
