@@ -141,8 +141,9 @@ static Config make_config() {
 }
 
 // Built configurations.  A 2-CTA tile spans 256 rows, which the contiguous
-// layout (128-row expert alignment) cannot guarantee to be one expert, so the
-// contiguous mode uses single-CTA tiles only.
+// layout (128-row expert alignment) cannot guarantee to be one expert; its
+// 2-CTA tiles pair blocks 2j and 2j+1 and run a second pass for the pairs
+// that straddle an expert boundary (at most one per expert).
 // Host-side id of the dense kernels with FP32 output (optionally + C).
 constexpr int MODE_DENSE_F32 = 3;
 
@@ -158,6 +159,7 @@ static const Config* config_table(int* count) {
   } else if constexpr (MODE == MODE_CONTIG) {
     static const Config table[] = {
         make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
+        make_config<224, 6, MODE, 2, false, 2>(),
     };
     *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
     return table;
@@ -207,7 +209,7 @@ static double config_rate(const Config& c) {
 }
 
 template <int MODE>
-static const Config* choose_config(long long rows_est, int N, int K, int sms) {
+static const Config* choose_config(long long rows_est, int N, int K, int sms, int groups = 1) {
   if (t_force_bn) return find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes);
   (void)K;
   int n = 0;
@@ -218,7 +220,8 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms) {
     const Config& c = t[i];
     if ((MODE == MODE_MASKED || MODE == MODE_DENSE_F32 || rows_est <= 128) && c.ctas != 1) continue;
     const long long tile_m = 128LL * c.ctas;
-    const long long m_tiles = (rows_est + tile_m - 1) / tile_m;
+    long long m_tiles = (rows_est + tile_m - 1) / tile_m;
+    if (MODE == MODE_CONTIG && c.ctas == 2) m_tiles += groups;  // second-pass pairs at expert boundaries
     const long long n_tiles = (N + c.bn - 1) / c.bn;
     const long long units = std::max(1, sms / c.ctas);
     const long long tiles = m_tiles * n_tiles;
@@ -511,7 +514,7 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
     c = choose_config<MODE_MASKED>(est, N, K, sms);
     if (c) tiles = static_cast<long long>(num_groups) * ((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   } else {
-    c = kind == 1 ? choose_config<MODE_CONTIG>(M, N, K, sms) : choose_config<MODE_DENSE>(M, N, K, sms);
+    c = kind == 1 ? choose_config<MODE_CONTIG>(M, N, K, sms, num_groups) : choose_config<MODE_DENSE>(M, N, K, sms);
     if (c) tiles = static_cast<long long>((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   }
   if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
@@ -713,7 +716,7 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const
   if (M_total == 0) return DG_OK;
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const Config* cfg = choose_config<MODE_CONTIG>(M_total, N, K, di.sms);
+  const Config* cfg = choose_config<MODE_CONTIG>(M_total, N, K, di.sms, num_groups);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
   if ((r = build_maps_cached(maps, cfg, a, b, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
@@ -722,7 +725,7 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const
   args.N = N;
   args.K = K;
   args.G = num_groups;
-  args.num_m_blocks = M_total / 128;
+  args.num_m_blocks = (M_total + 128 * cfg->ctas - 1) / (128 * cfg->ctas);  // 128-row blocks or block pairs
   args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
   args.raster_m = raster_group(args.num_m_blocks);
   args.m_indices = m_indices;

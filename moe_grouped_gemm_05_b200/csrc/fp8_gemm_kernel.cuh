@@ -169,19 +169,30 @@ __device__ __forceinline__ void wait_phase_drain(uint64_t* bar, uint32_t parity)
   }
 }
 
-template <int MODE>
+template <int MODE, int CTAS>
 __device__ __forceinline__ int total_tiles(const GemmArgs& p, const int* prefix) {
   if (MODE == MODE_MASKED) return prefix[p.G];
+  // contiguous pairs: a second pass for the pairs whose two blocks have different experts
+  if (MODE == MODE_CONTIG && CTAS == 2) return 2 * p.num_m_blocks * p.num_n_blocks;
   return p.num_m_blocks * p.num_n_blocks;
 }
 
 // Tile order: dense / contiguous use groups of `raster_m` M blocks swept
 // column by column, so concurrently running CTAs share A rows and B columns
 // in L2; masked runs expert by expert, N block by N block, M blocks fastest.
+// Contiguous 2-CTA tiles pair the 128-row blocks 2j and 2j+1: the first pass
+// (g = 0) computes pair j with the expert of block 2j, the second (g = 1)
+// only the pairs whose block 2j+1 has another expert, with that expert.
 template <int MODE, int TILE_M>
 __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* prefix,
                                         const int* counts) {
   Tile tl;
+  int pass = 0;
+  if (MODE == MODE_CONTIG && TILE_M == 256) {
+    const int per_pass = p.num_m_blocks * p.num_n_blocks;
+    pass = t >= per_pass ? 1 : 0;
+    t -= pass * per_pass;
+  }
   if (MODE == MODE_MASKED) {
     int g = 0;
     while (prefix[g + 1] <= t) ++g;
@@ -198,9 +209,23 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
     const int within = t - grp * per_group;
     tl.m_blk = first_m + within % gsize;
     tl.n_blk = within / gsize;
-    tl.g = 0;
+    tl.g = pass;
   }
   return tl;
+}
+
+// Expert of a contiguous-layout tile, or -1 when the tile has nothing to
+// compute: its (first) block starts with a padding row or an out-of-range
+// index, or it is a second-pass pair whose blocks share one expert.
+template <int CTAS>
+__device__ __forceinline__ int contig_expert(const Tile& tl, const GemmArgs& p) {
+  const int blocks = p.rows / 128;
+  const int blk = CTAS * tl.m_blk + tl.g;
+  if (blk >= blocks) return -1;
+  const int e = __ldg(&p.m_indices[blk * 128]);
+  if (e < 0 || e >= p.G) return -1;
+  if (CTAS == 2 && tl.g == 1 && __ldg(&p.m_indices[(blk - 1) * 128]) == e) return -1;
+  return e;
 }
 
 template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1>
@@ -295,7 +320,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   if constexpr (kPair) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const int ntiles = total_tiles<MODE>(p, prefix);
+  const int ntiles = total_tiles<MODE, CTAS>(p, prefix);
 
   if (warp == 0 || (PIPES == 2 && warp == 7)) {
     // ============================================================ producer
@@ -307,8 +332,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
       int grp_a = 0, grp_b = 0;
       if (MODE == MODE_CONTIG) {
-        const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
-        if (e < 0 || e >= p.G) continue;
+        const int e = contig_expert<CTAS>(tl, p);
+        if (e < 0) continue;
         grp_b = e;
       } else if (MODE == MODE_MASKED) {
         grp_a = grp_b = tl.g;
@@ -375,8 +400,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       for (int t = unit0; t < ntiles && ok; t += units) {
         if (MODE == MODE_CONTIG) {  // only the contiguous layout can skip a tile
           const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
-          const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
-          if (e < 0 || e >= p.G) continue;
+          if (contig_expert<CTAS>(tl, p) < 0) continue;
         }
         if (!take(li)) continue;
         // one pipeline: alternate accumulators; two: accumulator = pipeline
@@ -460,8 +484,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
       int grp_a = 0, grp_b = 0;
       if (MODE == MODE_CONTIG) {
-        const int e = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
-        if (e < 0 || e >= p.G) continue;
+        const int e = contig_expert<CTAS>(tl, p);
+        if (e < 0) continue;
         grp_b = e;
       } else if (MODE == MODE_MASKED) {
         grp_a = grp_b = tl.g;
@@ -531,14 +555,15 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     uint32_t local_tile = 0;
     for (int t = unit0; t < ntiles; t += units) {
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
-      int expert = 0;
+      int expert = 0, own_e = 0;
       if (MODE == MODE_CONTIG) {
-        expert = __ldg(&p.m_indices[tl.m_blk * L::kTileM]);
-        if (expert < 0 || expert >= p.G) {
-          if ((expert < -1 || expert >= p.G) && warp == 2 && lane == 0 && tl.n_blk == 0)
-            atomicOr(&g_dg_error, 0x2);
-          continue;
-        }
+        // expert of this CTA's own 128-row block (a pair's blocks may differ)
+        const int own_blk = CTAS * tl.m_blk + static_cast<int>(rank);
+        own_e = own_blk < p.rows / 128 ? __ldg(&p.m_indices[own_blk * 128]) : -1;
+        if ((own_e < -1 || own_e >= p.G) && warp == 2 && lane == 0 && tl.n_blk == 0 && tl.g == 0)
+          atomicOr(&g_dg_error, 0x2);
+        expert = contig_expert<CTAS>(tl, p);
+        if (expert < 0) continue;
       }
       const uint32_t acc = local_tile % L::kNumAcc;
       const uint32_t acc_use = local_tile / L::kNumAcc;
@@ -554,9 +579,10 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       if (MODE == MODE_DENSE) {
         valid = m_local < p.rows;
       } else if (MODE == MODE_CONTIG) {
-        const int idx = __ldg(&p.m_indices[m_local]);
-        valid = idx == expert;
-        if (!valid && idx != -1 && tl.n_blk == 0 && half == 0)
+        const int idx = m_local < p.rows ? __ldg(&p.m_indices[m_local]) : -1;
+        // rows of this CTA's block belong to the tile only when the block's expert is the tile's
+        valid = own_e == expert && idx == expert;
+        if (own_e == expert && idx != expert && idx != -1 && tl.n_blk == 0 && half == 0)
           atomicOr(&g_dg_error, (idx >= 0 && idx < p.G) ? 0x8 : 0x2);
       } else {
         valid = m_local < counts[tl.g];

@@ -16,6 +16,7 @@ pytestmark = pytest.mark.gpu
 # (block_n, ctas, pipes)
 BUILT = [(128, 1, 1), (224, 1, 1), (256, 1, 1), (128, 2, 1), (224, 2, 1), (256, 2, 1), (224, 2, 2), (128, 2, 2)]
 BUILT_1CTA = [c for c in BUILT if c[1] == 1]
+BUILT_CONTIG = BUILT_1CTA + [(224, 2, 2)]  # the contiguous layout's configurations
 SENTINEL = 0xDEAD
 
 
@@ -151,7 +152,7 @@ def test_dense_per_block_scales(cfg, lo, hi, exact):
 # ------------------------------------------------------------------ contiguous
 
 
-@pytest.mark.parametrize("cfg", BUILT_1CTA)
+@pytest.mark.parametrize("cfg", BUILT_CONTIG)
 def test_contiguous_small(cfg):
     p = synth.contiguous_problem(4, 512, 512, rows=0, seed=77, counts=[130, 0, 70, 250])
     sa, sb = packed(p)
@@ -164,6 +165,32 @@ def test_contiguous_small(cfg):
     assert oracle.m_grouped_fp8_gemm_nt_contiguous(p.a, sa, p.b, sb, p.m_indices, ref, p.G, p.N, p.K) == 0
     valid = p.m_indices >= 0
     check_close(got[valid], ref[valid], f"contiguous cfg={cfg}")
+    assert (got[~valid] == SENTINEL).all()
+    assert dg.get_device_error() == 0
+
+
+@pytest.mark.parametrize("cfg", BUILT_CONTIG)
+def test_contiguous_block_pairs_edge_layouts(cfg):
+    """Blocks of one pair with different experts, an all-padding block first in
+    a pair, a partly padded block, an expert repeated out of order and an odd
+    number of blocks: every valid row matches the oracle, no other row is written."""
+    layout = [(1, 128), (1, 60), (-1, 0), (0, 100), (2, 128), (2, 10), (0, 128)]  # (expert, rows) per block
+    m_idx = np.full(128 * len(layout), -1, np.int32)
+    for blk, (e, n) in enumerate(layout):
+        m_idx[128 * blk:128 * blk + n] = e
+    base = synth.contiguous_problem(3, 384, 384, rows=0, seed=78, counts=[128] * 7)
+    p = synth.Problem("contiguous", "pairs", base.a, base.sfa, base.b, base.sfb, len(m_idx), base.N, base.K, 3,
+                      m_indices=m_idx)
+    sa, sb = packed(p)
+    t = to_device(p, sa, sb)
+    dg.set_config(*cfg)
+    d = _sentinel((p.M, p.N))
+    dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], t["m_indices"], d)
+    got = bits(d)
+    ref = np.full((p.M, p.N), SENTINEL, np.uint16)
+    assert oracle.m_grouped_fp8_gemm_nt_contiguous(p.a, sa, p.b, sb, p.m_indices, ref, p.G, p.N, p.K) == 0
+    valid = p.m_indices >= 0
+    check_close(got[valid], ref[valid], f"contiguous pairs cfg={cfg}")
     assert (got[~valid] == SENTINEL).all()
     assert dg.get_device_error() == 0
 
