@@ -72,6 +72,29 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
                    int M, int N, int K, void* stream);
 
 /*
+ * Dense FP8 GEMM with the other operand layouts (the ssnai.com analysis,
+ * "SM90 vs SM100": SM100 serves NT, TN, NN and TT).  The first letter is the
+ * LHS, the second the RHS; N = not transposed, T = transposed, so NT is
+ * A [M][K] with B [N][K].  The product and the scales are those of
+ * dg_fp8_gemm_nt: D[m][n] = sum_k A(m,k) B(n,k) with A's 1x128 scales along
+ * K per row m and B's 128x128 block scales (same packed layouts).  Only the
+ * storage of the FP8 operands changes:
+ *   NN : a = A  as [M][K] (K contiguous),  b = B  as [K][N] (N contiguous)
+ *   TN : a = A  as [K][M] (M contiguous),  b = B  as [K][N] (N contiguous)
+ *   TT : a = A  as [K][M] (M contiguous),  b = B  as [N][K] (K contiguous)
+ * The tensor core reads the M- or N-contiguous tiles directly; nothing is
+ * transposed in memory.  Extra requirement: M % 16 == 0 when a is [K][M]
+ * (16-byte row stride).  Tiles: B stored [K][N] uses 128- or 256-wide N
+ * tiles.  Errors and ownership as dg_fp8_gemm_nt.
+ */
+int dg_fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream);
+int dg_fp8_gemm_tn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream);
+int dg_fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream);
+
+/*
  * Dense FP8 GEMM, NT layout, with the recipe and output options of DeepGEMM's
  * `fp8_gemm_nt(a, b, d, c=None, recipe=...)` (nightvoyager.top report, "解法哲学";
  * "1d1d / 1d2d" kernels under "关键设计决策"; the juejin.cn article §2.1's

@@ -18,6 +18,13 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libdg.so")
 HEADER = os.path.join(os.path.dirname(HERE), "include", "dg.h")
 
+DG_OK = 0
+DG_ERR_NULL = -1
+DG_ERR_SHAPE = -2
+DG_ERR_ALIGN = -3
+DG_ERR_UNSUPPORTED = -4
+DG_ERR_CUDA = -5
+
 DG_DEVERR_BAD_SCALE = 0x1
 DG_DEVERR_BAD_EXPERT = 0x2
 DG_DEVERR_BAD_MASKED_M = 0x4
@@ -43,6 +50,8 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32p, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
     lib.dg_fp8_gemm_nt.argtypes = [vp, i32p, vp, i32p, vp, i, i, i, vp]
+    for name in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
+        getattr(lib, name).argtypes = [vp, i32p, vp, i32p, vp, i, i, i, vp]
     lib.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
     lib.dg_m_grouped_fp8_gemm_nt_masked.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
     lib.dg_pack_sf_ue8m0.argtypes = [vp, i32p, i, i, i, vp]
@@ -163,6 +172,32 @@ def fp8_gemm_nt(a, sfa, b, sfb, d=None) -> torch.Tensor:
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
         raise ValueError("d must be a contiguous bf16 [M, N] tensor")
     _check(load().dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    return d
+
+
+def fp8_gemm(layout: str, a, sfa, b, sfb, d=None) -> torch.Tensor:
+    """D[M,N] (bf16) = A . B^T with the operands stored in `layout` ("nt", "nn", "tn" or "tt").
+
+    First letter LHS, second RHS, N = not transposed, T = transposed:
+    a is A [M,K] for "n?" and A^T [K,M] for "t?"; b is B [N,K] for "?t" and B^T [K,N] for "?n".
+    """
+    if layout not in ("nt", "nn", "tn", "tt"):
+        raise ValueError(f"unknown layout {layout!r}")
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb")
+    if not (a.is_contiguous() and b.is_contiguous()):
+        raise ValueError("a and b must be contiguous")
+    K, M = a.shape if layout[0] == "t" else a.shape[::-1]
+    K2, N = b.shape if layout[1] == "n" else b.shape[::-1]
+    if K2 != K:
+        raise ValueError("a and b disagree on K")
+    if tuple(sfa.shape) != packed_sf_words(M, K // 128) or tuple(sfb.shape) != packed_sf_words(-(-N // 128), K // 128):
+        raise ValueError("packed scale shapes do not match [ceil(Kb/4), align4(MN)]")
+    if d is None:
+        d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
+        raise ValueError("d must be a contiguous bf16 [M, N] tensor")
+    fn = getattr(load(), f"dg_fp8_gemm_{layout}")
+    _check(fn(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
     return d
 
 

@@ -122,21 +122,23 @@ struct Config {
   int smem = 0;
   int num_acc = 1;
   int pipes = 1;  // load/MMA pipelines per CTA (alternate tiles)
+  int layout = 0; // bit 0: A MN-major, bit 1: B MN-major
   int threads = kThreads;
   KernelFn fn = nullptr;
 };
 
-template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0>
 static Config make_config() {
   Config c;
   c.bn = BN;
   c.stages = STAGES;
   c.ctas = CTAS;
-  c.smem = Layout<BN, STAGES, CTAS, PIPES>::kSmemBytes;
-  c.num_acc = Layout<BN, STAGES, CTAS, PIPES>::kNumAcc;
+  c.smem = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>::kSmemBytes;
+  c.num_acc = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>::kNumAcc;
   c.pipes = PIPES;
+  c.layout = LAYOUT;
   c.threads = kThreadsFor<PIPES>;
-  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES>);
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES, LAYOUT>);
   return c;
 }
 
@@ -146,6 +148,9 @@ static Config make_config() {
 // that straddle an expert boundary (at most one per expert).
 // Host-side id of the dense kernels with FP32 output (optionally + C).
 constexpr int MODE_DENSE_F32 = 3;
+// Host-side ids of the dense kernels with MN-major operands: MODE_DENSE_MN + LAYOUT - 1
+// (LAYOUT 1: A MN-major (TT), 2: B MN-major (NN), 3: both (TN)).
+constexpr int MODE_DENSE_MN = 4;
 
 template <int MODE>
 static const Config* config_table(int* count) {
@@ -153,6 +158,22 @@ static const Config* config_table(int* count) {
     static const Config table[] = {
         make_config<128, 6, MODE_DENSE, 1, true>(), make_config<224, 4, MODE_DENSE, 1, true>(),
         make_config<256, 4, MODE_DENSE, 1, true>(),
+    };
+    *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
+    return table;
+  } else if constexpr (MODE == MODE_DENSE_MN) {
+    static const Config table[] = {
+        make_config<128, 6, MODE_DENSE, 1, false, 1, 1>(), make_config<224, 4, MODE_DENSE, 1, false, 1, 1>(),
+        make_config<224, 6, MODE_DENSE, 2, false, 2, 1>(),
+    };
+    *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
+    return table;
+  } else if constexpr (MODE == MODE_DENSE_MN + 1 || MODE == MODE_DENSE_MN + 2) {
+    // an MN-major B tile is whole 128-column boxes per CTA: 128 or 256 wide, 256 on a pair
+    constexpr int LAYOUT = MODE - MODE_DENSE_MN + 1;
+    static const Config table[] = {
+        make_config<128, 6, MODE_DENSE, 1, false, 1, LAYOUT>(), make_config<256, 4, MODE_DENSE, 1, false, 1, LAYOUT>(),
+        make_config<256, 6, MODE_DENSE, 2, false, 1, LAYOUT>(),
     };
     *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
     return table;
@@ -210,7 +231,10 @@ static double config_rate(const Config& c) {
 
 template <int MODE>
 static const Config* choose_config(long long rows_est, int N, int K, int sms, int groups = 1) {
-  if (t_force_bn) return find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes);
+  if (t_force_bn) {
+    if (const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes)) return f;
+    if (MODE < MODE_DENSE_MN) return nullptr;  // layouts build fewer tiles: fall back to the heuristic
+  }
   (void)K;
   int n = 0;
   const Config* t = config_table<MODE>(&n);
@@ -311,18 +335,29 @@ static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const Ge
 
 // Builds the tensor maps of one call.
 //   A : [GA][rowsA][K] bytes    box 128 x 128 (K x rows), 128-byte swizzle
+//       ([GA][K][rowsA] when MN-major: box 128 x 128 (rows x K))
 //   B : [GB][N][K] bytes        box 128 x BN/CTAS,         128-byte swizzle
+//       ([GB][K][N] when MN-major: box 128 x 128 (N x K), BN/CTAS/128 boxes per stage)
 //   D : [GD][rowsD][N] bf16     box 32 x 32,               64-byte swizzle
 static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const void* b, void* d,
                       int rowsA, int GA, int N, int K, int GB, int rowsD, int GD, bool d_f32 = false) {
   int r;
-  if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, rowsA, GA, K,
-                    static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A")))
+  if (cfg->layout & 1) {  // A stored [GA][K][rowsA]: 128 rows x 128 K per box
+    if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, rowsA, K, GA, rowsA,
+                      static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A")))
+      return r;
+  } else if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, rowsA, GA, K,
+                           static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A"))) {
     return r;
-  if ((r = make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K, N, GB, K,
-                    static_cast<uint64_t>(N) * K, 128, cfg->bn / cfg->ctas, CU_TENSOR_MAP_SWIZZLE_128B,
-                    "B")))
+  }
+  if (cfg->layout & 2) {  // B stored [GB][K][N]: 128 columns x 128 K per box
+    if ((r = make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, b, N, K, GB, N, static_cast<uint64_t>(N) * K, 128,
+                      128, CU_TENSOR_MAP_SWIZZLE_128B, "B")))
+      return r;
+  } else if ((r = make_map(&maps[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, b, K, N, GB, K, static_cast<uint64_t>(N) * K,
+                           128, cfg->bn / cfg->ctas, CU_TENSOR_MAP_SWIZZLE_128B, "B"))) {
     return r;
+  }
   if (d_f32) {  // 16 FP32 columns (64 B) per box row
     if ((r = make_map(&maps[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, d, N, rowsD, GD, static_cast<uint64_t>(N) * 4,
                       static_cast<uint64_t>(rowsD) * N * 4, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B, "D")))
@@ -459,6 +494,36 @@ __global__ void pack_sf_ue8m0_kernel(const float* __restrict__ sf, uint32_t* __r
 using namespace dg;
 
 // ==================================================================== C ABI
+
+template <int HMODE>
+static int gemm_dense(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
+                      int N, int K, void* stream) {
+  int r = check_common(a, sfa, b, sfb, d, N, K);
+  if (r) return r;
+  if (M < 0) return fail(DG_ERR_SHAPE, "M=%d must be >= 0", M);
+  if (M == 0) return DG_OK;
+  if (HMODE == MODE_DENSE_MN || HMODE == MODE_DENSE_MN + 2) {
+    if (M % 16 != 0) return fail(DG_ERR_SHAPE, "M=%d must be a multiple of 16 when A is stored K x M", M);
+  }
+  DeviceInfo di;
+  if ((r = device_info(&di))) return r;
+  const Config* cfg = choose_config<HMODE>(M, N, K, di.sms);
+  if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
+  CUtensorMap maps[3];
+  if ((r = build_maps_cached(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1))) return r;
+  GemmArgs args = {};
+  args.rows = M;
+  args.N = N;
+  args.K = K;
+  args.G = 1;
+  args.num_m_blocks = (M + 128 * cfg->ctas - 1) / (128 * cfg->ctas);
+  args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
+  args.raster_m = raster_group(args.num_m_blocks);
+  args.d = static_cast<__nv_bfloat16*>(d);
+  fill_scale_args(&args, sfa, sfb, M, N, K);
+  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
+  return launch<HMODE>(cfg, grid_size(di.sms, tiles, cfg), maps, args, static_cast<cudaStream_t>(stream));
+}
 
 extern "C" {
 
@@ -643,29 +708,22 @@ int dg_moe_unpermute_combine(const void* d_perm, const int32_t* row_of, const fl
 
 int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
                    int M, int N, int K, void* stream) {
-  int r = check_common(a, sfa, b, sfb, d, N, K);
-  if (r) return r;
-  if (M < 0) return fail(DG_ERR_SHAPE, "M=%d must be >= 0", M);
-  if (M == 0) return DG_OK;
-  DeviceInfo di;
-  if ((r = device_info(&di))) return r;
-  const Config* cfg = choose_config<MODE_DENSE>(M, N, K, di.sms);
-  if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
-  CUtensorMap maps[3];
-  if ((r = build_maps_cached(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1))) return r;
-  GemmArgs args = {};
-  args.rows = M;
-  args.N = N;
-  args.K = K;
-  args.G = 1;
-  args.num_m_blocks = (M + 128 * cfg->ctas - 1) / (128 * cfg->ctas);
-  args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
-  args.raster_m = raster_group(args.num_m_blocks);
-  args.d = static_cast<__nv_bfloat16*>(d);
-  fill_scale_args(&args, sfa, sfb, M, N, K);
-  const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
-  return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles, cfg), maps, args,
-                            static_cast<cudaStream_t>(stream));
+  return gemm_dense<MODE_DENSE>(a, sfa, b, sfb, d, M, N, K, stream);
+}
+
+int dg_fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream) {
+  return gemm_dense<MODE_DENSE_MN + 1>(a, sfa, b, sfb, d, M, N, K, stream);
+}
+
+int dg_fp8_gemm_tn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream) {
+  return gemm_dense<MODE_DENSE_MN + 2>(a, sfa, b, sfb, d, M, N, K, stream);
+}
+
+int dg_fp8_gemm_tt(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
+                   int M, int N, int K, void* stream) {
+  return gemm_dense<MODE_DENSE_MN>(a, sfa, b, sfb, d, M, N, K, stream);
 }
 
 int dg_fp8_gemm_nt_ex(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, const float* c,

@@ -37,7 +37,15 @@
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of
 // tile i overlaps the MMAs of tile i+1.
 //
-// PIPES = 2 (1-CTA tiles): every tcgen05 instruction costs its issuing thread
+// LAYOUT (dense only): bit 0 set = A stored K x M (MN-major), bit 1 set = B
+// stored K x N (MN-major); the pages' NT / NN / TN / TT layouts are LAYOUT
+// 0 / 2 / 3 / 1.  An MN-major operand is loaded as 128 x 128 TMA boxes whose
+// 128-byte rows run along M (or N) and read by the tensor core through an
+// MN-major descriptor: 128-byte swizzle atoms of 8 K-rows, SBO = 1024 B
+// between atoms along K, LBO = 16 KB between 128-wide atoms along M/N.
+// Each CTA's share of an MN-major B tile is a whole number of 128 columns.
+//
+// PIPES = 2: every tcgen05 instruction costs its issuing thread
 // a fixed ~60-70 cycles, so one thread issuing the 4 MMAs + commit of a
 // 128x224x128 K block spends ~300 of the block's 448 tensor-pipe cycles on
 // issue alone and, with its waits, cannot keep the pipe busy.  The cost is
@@ -89,8 +97,9 @@ struct GemmArgs {
   const float* c;     // optional FP32 addend [rows][N] (OUT_F32 only), nullptr for none
 };
 
-template <int BN, int STAGES, int CTAS, int PIPES = 1>
+template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0>
 struct Layout {
+  static_assert(!(LAYOUT & 2) || (BN / CTAS) % 128 == 0, "an MN-major B tile is whole 128-column boxes per CTA");
   static_assert(CTAS == 1 || CTAS == 2, "CTAS is 1 or 2");
   static_assert(PIPES == 1 || (PIPES == 2 && STAGES % 2 == 0), "two pipelines need an even number of stages");
   static constexpr int kStagesPer = STAGES / PIPES;     // stages of each pipeline's ring
@@ -228,11 +237,14 @@ __device__ __forceinline__ int contig_expert(const Tile& tl, const GemmArgs& p) 
   return e;
 }
 
-template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0>
 __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
-  using L = Layout<BN, STAGES, CTAS, PIPES>;
+  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>;
+  static_assert(LAYOUT == 0 || MODE == MODE_DENSE, "MN-major operands are built for the dense GEMM only");
+  constexpr bool kAmn = (LAYOUT & 1) != 0;
+  constexpr bool kBmn = (LAYOUT & 2) != 0;
   constexpr bool kPair = CTAS == 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -350,12 +362,21 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
           uint8_t* a_dst = smem + L::kOffA + s * L::kABytes;
           uint8_t* b_dst = smem + L::kOffB + s * L::kBBytes;
           const int b_row = n0 + static_cast<int>(rank) * L::kBRows;
-          if constexpr (kPair) {
-            tma_load_3d_pair(a_dst, &tm_a, full0 + 8 * s, kb * kBK, m_base, grp_a);
-            tma_load_3d_pair(b_dst, &tm_b, full0 + 8 * s, kb * kBK, b_row, grp_b);
+          // K-major boxes are (K, rows); MN-major boxes are (rows, K), 128 x 128 each
+          const int ax = kAmn ? m_base : kb * kBK, ay = kAmn ? kb * kBK : m_base;
+          if constexpr (kPair) tma_load_3d_pair(a_dst, &tm_a, full0 + 8 * s, ax, ay, grp_a);
+          else tma_load_3d(a_dst, &tm_a, &full_bar[s], ax, ay, grp_a);
+          if constexpr (kBmn) {
+#pragma unroll
+            for (int j = 0; j < L::kBRows / 128; ++j) {
+              if constexpr (kPair)
+                tma_load_3d_pair(b_dst + j * 128 * kBK, &tm_b, full0 + 8 * s, b_row + 128 * j, kb * kBK, grp_b);
+              else
+                tma_load_3d(b_dst + j * 128 * kBK, &tm_b, &full_bar[s], b_row + 128 * j, kb * kBK, grp_b);
+            }
           } else {
-            tma_load_3d(a_dst, &tm_a, &full_bar[s], kb * kBK, m_base, grp_a);
-            tma_load_3d(b_dst, &tm_b, &full_bar[s], kb * kBK, b_row, grp_b);
+            if constexpr (kPair) tma_load_3d_pair(b_dst, &tm_b, full0 + 8 * s, kb * kBK, b_row, grp_b);
+            else tma_load_3d(b_dst, &tm_b, &full_bar[s], kb * kBK, b_row, grp_b);
           }
         }
         if (lane == 0) {
@@ -381,12 +402,17 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     // are precomputed, stage/phase counters are incremental and barrier polls
     // take an inline fast path.
     if ((!kPair || rank == 0) && lane == 0) {
-      const uint32_t a_lo0 =
-          static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffA + sbase * L::kABytes), 16, 1024, 2));
-      const uint32_t b_lo0 =
-          static_cast<uint32_t>(make_smem_desc(smem_u32(smem + L::kOffB + sbase * L::kBBytes), 16, 1024, 2));
+      // LBO only matters for MN-major operands (16 KB between 128-wide boxes);
+      // it sits in the low word, SBO (1024 B: 8 rows of 128 B) in the high word
+      const uint32_t a_lo0 = static_cast<uint32_t>(
+          make_smem_desc(smem_u32(smem + L::kOffA + sbase * L::kABytes), kAmn ? 128 * kBK : 16, 1024, 2));
+      const uint32_t b_lo0 = static_cast<uint32_t>(
+          make_smem_desc(smem_u32(smem + L::kOffB + sbase * L::kBBytes), kBmn ? 128 * kBK : 16, 1024, 2));
       const uint32_t desc_hi = static_cast<uint32_t>(make_smem_desc(0, 16, 1024, 2) >> 32);
-      const uint32_t idesc0 = make_idesc_mxf8(L::kTileM, BN, 0, 0);
+      const uint32_t idesc0 = make_idesc_mxf8(L::kTileM, BN, 0, 0, kAmn, kBmn);
+      // start-address step per K = 32 (address field in 16-byte units): K-major,
+      // +32 B inside the swizzled 128-byte row; MN-major, +4 atoms of 8 K-rows
+      constexpr uint32_t kAStep = kAmn ? 256 : 2, kBStep = kBmn ? 256 : 2;
       constexpr uint32_t kSfIdStep = (1u << 4) | (1u << 29);  // +1 in both scale-factor byte selectors
       const uint32_t full_base = smem_u32(full_bar + sbase);
       const uint32_t empty_base = smem_u32(empty_bar + sbase);
@@ -447,11 +473,10 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
               }
               const uint64_t a_desc = (static_cast<uint64_t>(desc_hi) << 32) | (a_lo0 + s * (L::kABytes >> 4));
               const uint64_t b_desc = (static_cast<uint64_t>(desc_hi) << 32) | (b_lo0 + s * (L::kBBytes >> 4));
-              // +32 bytes along K inside the 128-byte swizzled row = +2 in the address field
               mma_mxf8f6f4<CTAS>(d_tmem, a_desc, b_desc, id, sf_col, sf_col + 4, accumulate);
-              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2, b_desc + 2, id, sf_col, sf_col + 4, 1u);
-              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 4, b_desc + 4, id, sf_col, sf_col + 4, 1u);
-              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 6, b_desc + 6, id, sf_col, sf_col + 4, 1u);
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + kAStep, b_desc + kBStep, id, sf_col, sf_col + 4, 1u);
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 2 * kAStep, b_desc + 2 * kBStep, id, sf_col, sf_col + 4, 1u);
+              mma_mxf8f6f4<CTAS>(d_tmem, a_desc + 3 * kAStep, b_desc + 3 * kBStep, id, sf_col, sf_col + 4, 1u);
               accumulate = 1;
               if constexpr (kPair) tc_commit_pair_addr(empty_base + 8 * s);
               else tc_commit_addr<1>(empty_base + 8 * s);

@@ -353,12 +353,14 @@ __device__ __forceinline__ uint64_t make_smem_desc(uint32_t saddr, uint32_t lbo_
 }
 
 // Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 x E4M3,
-// both K-major, UE8M0 scale type, MMA shape M x N, scale-factor byte selectors.
+// UE8M0 scale type, MMA shape M x N, scale-factor byte selectors, and the
+// major-ness of A and B in shared memory (0: K-major, 1: MN-major).
 __host__ __device__ constexpr uint32_t make_idesc_mxf8(uint32_t M, uint32_t N, uint32_t sfa_id,
-                                                       uint32_t sfb_id) {
+                                                       uint32_t sfb_id, uint32_t a_mn = 0,
+                                                       uint32_t b_mn = 0) {
   return ((sfb_id & 3u) << 4)        // B scale-factor byte selector
          | (0u << 7) | (0u << 10)    // A, B formats: E4M3
-         | (0u << 15) | (0u << 16)   // A, B K-major
+         | ((a_mn & 1u) << 15) | ((b_mn & 1u) << 16)  // A, B major-ness
          | ((N >> 3) << 17)          // N / 8
          | (1u << 23)                // scale type UE8M0
          | ((M >> 4) << 24)          // M / 16
