@@ -215,6 +215,13 @@ int dg_get_device_error(void* stream, int* err);
 int dg_set_num_sms(int n);
 int dg_get_num_sms(void);
 
+/* Programmatic dependent launch for every kernel of this library (on by
+ * default): a kernel's set-up (barrier init, tensor-memory allocation) may
+ * overlap the end of the previous kernel on the stream; the kernel waits for
+ * that kernel's completion before its first global-memory access, so stream
+ * order is kept.  enable = 0 launches plainly.  Returns the previous setting. */
+int dg_set_pdl(int enable);
+
 /* Forces the tile configuration of the next calls on this host thread:
  * block_n (a built N tile width), ctas (1: 128-row tiles on one SM;
  * 2: 256-row tiles on a pair of SMs; 0: whichever is built, 1 first) and

@@ -65,6 +65,7 @@ def load() -> ctypes.CDLL:
     lib.dg_get_mk_alignment_for_contiguous_layout.argtypes = []
     lib.dg_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.dg_set_num_sms.argtypes = [i]
+    lib.dg_set_pdl.argtypes = [i]
     lib.dg_get_num_sms.argtypes = []
     lib.dg_set_config.argtypes = [i, i, i]
     lib.dg_describe_config.argtypes = [i, i, i, i, i, ctypes.c_char_p, i]
@@ -117,8 +118,8 @@ def packed_sf_words(mn: int, kb: int) -> tuple[int, int]:
     return (kb + 3) // 4, (mn + 3) // 4 * 4
 
 
-def pack_sf_ue8m0(sf: torch.Tensor) -> torch.Tensor:
-    """fp32 power-of-two scales [batch?, mn, kb] -> int32 [batch?, ceil(kb/4), align4(mn)]."""
+def pack_sf_ue8m0(sf: torch.Tensor, out=None) -> torch.Tensor:
+    """fp32 power-of-two scales [batch?, mn, kb] -> int32 [batch?, ceil(kb/4), align4(mn)] (into `out` if given)."""
     if sf.dtype != torch.float32 or not sf.is_cuda or not sf.is_contiguous():
         raise TypeError("sf must be a contiguous float32 CUDA tensor")
     squeeze = sf.dim() == 2
@@ -127,9 +128,14 @@ def pack_sf_ue8m0(sf: torch.Tensor) -> torch.Tensor:
         raise ValueError("sf must be [mn, kb] or [batch, mn, kb]")
     batch, mn, kb = s3.shape
     kp, mn4 = packed_sf_words(mn, kb)
-    out = torch.empty((batch, kp, mn4), dtype=torch.int32, device=sf.device)
+    if out is None:
+        out = torch.empty((batch, kp, mn4), dtype=torch.int32, device=sf.device)
+    elif out.dtype != torch.int32 or not out.is_contiguous() or out.numel() != batch * kp * mn4:
+        raise ValueError("out must be a contiguous int32 tensor of the packed shape")
     _check(load().dg_pack_sf_ue8m0(_ptr(s3), _ptr(out), batch, mn, kb, _stream()))
-    return out[0] if squeeze else out
+    if out.dim() == 3 and squeeze:
+        return out[0]
+    return out
 
 
 def quantize_fp8_1x128(x: torch.Tensor, q=None, sf=None):
@@ -254,11 +260,12 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m, d=None) -> torch.Tens
     return d
 
 
-def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: torch.Tensor):
+def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: torch.Tensor, out=None):
     """Contiguous-layout permutation of routed tokens.
 
     Returns a dict with a (float8 [M_cap, K]), sfa (int32 [kp, M_cap]), m_indices, src_of ([M_cap]) and
     row_of ([T, topk]); a / sfa / m_indices are the operands of m_grouped_fp8_gemm_nt_contiguous.
+    `out`, if given, is such a dict of preallocated tensors (M_cap = dg_moe_permute_capacity).
     """
     _i32(topk_ids, "topk_ids"), _fp8(q, "q"), _i32(sfa, "sfa")
     T, topk = topk_ids.shape
@@ -268,13 +275,19 @@ def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: 
         _check(cap)
     kp = (K // 128 + 3) // 4
     dev = q.device
-    out = {
-        "a": torch.empty((cap, K), dtype=torch.float8_e4m3fn, device=dev),
-        "sfa": torch.empty((kp, cap), dtype=torch.int32, device=dev),
-        "m_indices": torch.empty((cap,), dtype=torch.int32, device=dev),
-        "src_of": torch.empty((cap,), dtype=torch.int32, device=dev),
-        "row_of": torch.empty((T, topk), dtype=torch.int32, device=dev),
-    }
+    if out is None:
+        out = {
+            "a": torch.empty((cap, K), dtype=torch.float8_e4m3fn, device=dev),
+            "sfa": torch.empty((kp, cap), dtype=torch.int32, device=dev),
+            "m_indices": torch.empty((cap,), dtype=torch.int32, device=dev),
+            "src_of": torch.empty((cap,), dtype=torch.int32, device=dev),
+            "row_of": torch.empty((T, topk), dtype=torch.int32, device=dev),
+        }
+    else:
+        want = {"a": (cap, K), "sfa": (kp, cap), "m_indices": (cap,), "src_of": (cap,), "row_of": (T, topk)}
+        for key, shape in want.items():
+            if key not in out or tuple(out[key].shape) != shape or not out[key].is_contiguous():
+                raise ValueError(f"out[{key!r}] must be a contiguous tensor of shape {shape}")
     _check(load().dg_moe_permute(_ptr(topk_ids), T, topk, num_experts, _ptr(q), _ptr(sfa), K, _ptr(out["a"]),
                                  _ptr(out["sfa"]), _ptr(out["m_indices"]), _ptr(out["row_of"]), _ptr(out["src_of"]),
                                  cap, _stream()))
@@ -306,6 +319,11 @@ def get_device_error() -> int:
 
 def set_num_sms(n: int) -> int:
     return load().dg_set_num_sms(n)
+
+
+def set_pdl(enable: bool) -> bool:
+    """Programmatic dependent launch on/off for the library's kernels; returns the previous setting."""
+    return bool(load().dg_set_pdl(1 if enable else 0))
 
 
 def set_config(block_n: int, ctas: int = 0, pipes: int = 0) -> None:

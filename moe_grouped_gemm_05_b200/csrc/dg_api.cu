@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -44,6 +45,46 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // ------------------------------------------------------------------ device info
 
 static int g_num_sms_override = 0;
+// Programmatic dependent launch of every kernel (on by default): a kernel may
+// start its set-up while the previous grid of the stream finishes, and waits
+// (griddepcontrol.wait) before its first global-memory access.
+static std::atomic<int> g_pdl{1};
+
+// One launch attribute set: programmatic stream serialisation when enabled,
+// plus a cluster of `cluster` CTAs along x when cluster > 1.
+struct LaunchAttrs {
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  explicit LaunchAttrs(int cluster) {
+    if (g_pdl.load(std::memory_order_relaxed)) {
+      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
+    }
+    if (cluster > 1) {
+      attr[n].id = cudaLaunchAttributeClusterDimension;
+      attr[n].val.clusterDim.x = cluster;
+      attr[n].val.clusterDim.y = 1;
+      attr[n].val.clusterDim.z = 1;
+      ++n;
+    }
+  }
+};
+
+// cudaLaunchKernelEx of a plain (non-cluster) kernel with the PDL attribute.
+template <typename... Params, typename... Args>
+static cudaError_t launch_plain(void (*kernel)(Params...), long long blocks, int threads, cudaStream_t st,
+                                Args&&... args) {
+  LaunchAttrs la(1);
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3(static_cast<unsigned>(blocks));
+  lc.blockDim = dim3(threads);
+  lc.dynamicSmemBytes = 0;
+  lc.stream = st;
+  lc.attrs = la.attr;
+  lc.numAttrs = la.n;
+  return cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+}
 static thread_local int t_force_bn = 0;
 
 struct DeviceInfo {
@@ -123,11 +164,13 @@ struct Config {
   int num_acc = 1;
   int pipes = 1;  // load/MMA pipelines per CTA (alternate tiles)
   int layout = 0; // bit 0: A MN-major, bit 1: B MN-major
+  bool splitk = false;  // both pipelines on every tile, each on half of K
   int threads = kThreads;
   KernelFn fn = nullptr;
 };
 
-template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0,
+          bool SPLITK = false>
 static Config make_config() {
   Config c;
   c.bn = BN;
@@ -137,8 +180,9 @@ static Config make_config() {
   c.num_acc = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>::kNumAcc;
   c.pipes = PIPES;
   c.layout = LAYOUT;
+  c.splitk = SPLITK;
   c.threads = kThreadsFor<PIPES>;
-  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES, LAYOUT>);
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES, LAYOUT, SPLITK>);
   return c;
 }
 
@@ -189,6 +233,8 @@ static const Config* config_table(int* count) {
         make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
         make_config<128, 6, MODE, 2>(), make_config<224, 6, MODE, 2>(), make_config<256, 6, MODE, 2>(),
         make_config<224, 6, MODE, 2, false, 2>(), make_config<128, 6, MODE, 2, false, 2>(),
+        make_config<64, 8, MODE, 1>(), make_config<64, 6, MODE, 1, false, 2, 0, true>(),
+        make_config<128, 4, MODE, 1, false, 2, 0, true>(),
     };
     *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
     return table;
@@ -243,6 +289,9 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms, in
   for (int i = 0; i < n; ++i) {
     const Config& c = t[i];
     if ((MODE == MODE_MASKED || MODE == MODE_DENSE_F32 || rows_est <= 128) && c.ctas != 1) continue;
+    // split-K tiles keep no second accumulator for overlap: only for a single M block
+    // (decode), and only when K has at least two groups of 4 K blocks
+    if (c.splitk && (rows_est > 128 || K <= 4 * 128)) continue;
     const long long tile_m = 128LL * c.ctas;
     long long m_tiles = (rows_est + tile_m - 1) / tile_m;
     if (MODE == MODE_CONTIG && c.ctas == 2) m_tiles += groups;  // second-pass pairs at expert boundaries
@@ -252,7 +301,7 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms, in
     const long long waves = (tiles + units - 1) / units;
     // padded work in units of 128x128 tile-K-blocks, spread over the whole grid
     const double work = static_cast<double>(waves) * units * (tile_m / 128.0) * (c.bn / 128.0);
-    const double cost = work / config_rate(c);
+    const double cost = work / config_rate(c) * (c.splitk ? 0.5 : 1.0);  // split-K halves the K loop
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = &c;
@@ -315,20 +364,14 @@ static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const Ge
       attr_done[idx] = true;
     }
   }
+  LaunchAttrs la(cfg->ctas);
   cudaLaunchConfig_t lc = {};
-  cudaLaunchAttribute attr[1];
   lc.gridDim = dim3(grid);
   lc.blockDim = dim3(cfg->threads);
   lc.dynamicSmemBytes = cfg->smem;
   lc.stream = stream;
-  if (cfg->ctas == 2) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    lc.attrs = attr;
-    lc.numAttrs = 1;
-  }
+  lc.attrs = la.attr;
+  lc.numAttrs = la.n;
   DG_CUDA_TRY(cudaLaunchKernelEx(&lc, cfg->fn, maps[0], maps[1], maps[2], args));
   return DG_OK;
 }
@@ -456,6 +499,8 @@ static int grid_size(int sms, long long tiles, const Config* cfg) {
 
 __global__ void pack_sf_ue8m0_kernel(const float* __restrict__ sf, uint32_t* __restrict__ out,
                                      int batch, int mn, int kb, int kp, int mn4) {
+  grid_dep_wait();
+  grid_dep_launch();
   const long long total = static_cast<long long>(batch) * kp * mn4;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
@@ -542,6 +587,8 @@ int dg_set_num_sms(int n) {
   return prev;
 }
 
+int dg_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0); }
+
 int dg_get_num_sms(void) {
   DeviceInfo di;
   if (device_info(&di) != DG_OK) return g_num_sms_override;
@@ -583,8 +630,8 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
     if (c) tiles = static_cast<long long>((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   }
   if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
-  snprintf(buf, buflen, "%dx%dx%d%s%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
-           c->pipes == 2 ? "(2pipe)" : "", grid_size(sms, tiles, c));
+  snprintf(buf, buflen, "%dx%dx%d%s%s%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
+           c->pipes == 2 ? "(2pipe)" : "", c->splitk ? "(splitk)" : "", grid_size(sms, tiles, c));
   return DG_OK;
 }
 
@@ -613,9 +660,8 @@ int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb
   if (r) return r;
   const int threads = 256;
   const long long blocks = std::min<long long>((total + threads - 1) / threads, 8LL * di.sms);
-  pack_sf_ue8m0_kernel<<<static_cast<int>(blocks), threads, 0, static_cast<cudaStream_t>(stream)>>>(
-      sf, reinterpret_cast<uint32_t*>(packed), batch, mn, kb, kp, mn4);
-  DG_CUDA_TRY(cudaGetLastError());
+  DG_CUDA_TRY(launch_plain(pack_sf_ue8m0_kernel, blocks, threads, static_cast<cudaStream_t>(stream), sf,
+                           reinterpret_cast<uint32_t*>(packed), batch, mn, kb, kp, mn4));
   return DG_OK;
 }
 
@@ -637,14 +683,12 @@ int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int 
   const long long blocks = std::min<long long>((units + 7) / 8, 32LL * di.sms);
   auto st = static_cast<cudaStream_t>(stream);
   if (x_dtype == 0)
-    quantize_1x128_kernel<__nv_bfloat16><<<static_cast<int>(blocks), threads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(q), reinterpret_cast<uint32_t*>(sf), batch, M,
-        K, kp, mn4);
+    DG_CUDA_TRY(launch_plain(quantize_1x128_kernel<__nv_bfloat16>, blocks, threads, st,
+                             static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(q),
+                             reinterpret_cast<uint32_t*>(sf), batch, M, K, kp, mn4));
   else
-    quantize_1x128_kernel<float><<<static_cast<int>(blocks), threads, 0, st>>>(
-        static_cast<const float*>(x), static_cast<uint8_t*>(q), reinterpret_cast<uint32_t*>(sf), batch, M, K, kp,
-        mn4);
-  DG_CUDA_TRY(cudaGetLastError());
+    DG_CUDA_TRY(launch_plain(quantize_1x128_kernel<float>, blocks, threads, st, static_cast<const float*>(x),
+                             static_cast<uint8_t*>(q), reinterpret_cast<uint32_t*>(sf), batch, M, K, kp, mn4));
   return DG_OK;
 }
 
@@ -676,16 +720,14 @@ int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, co
   int r = device_info(&di);
   if (r) return r;
   auto st = static_cast<cudaStream_t>(stream);
-  moe_route_kernel<<<num_experts, kMoeThreads, 0, st>>>(topk_ids, static_cast<int>(n), topk, num_experts, M_cap,
-                                                        m_indices, row_of, src_of);
-  DG_CUDA_TRY(cudaGetLastError());
+  DG_CUDA_TRY(launch_plain(moe_route_kernel, num_experts, kMoeThreads, st, topk_ids, static_cast<int>(n), topk,
+                           num_experts, M_cap, m_indices, row_of, src_of));
   const int kp = (K / 128 + 3) / 4;
   const long long work = static_cast<long long>(M_cap) * (K / 16);
   const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 16LL * di.sms));
-  moe_gather_kernel<<<static_cast<int>(blocks), 256, 0, st>>>(
-      static_cast<const uint8_t*>(q), reinterpret_cast<const uint32_t*>(sfa), T, K, kp, src_of, M_cap,
-      static_cast<uint8_t*>(a_perm), reinterpret_cast<uint32_t*>(sfa_perm));
-  DG_CUDA_TRY(cudaGetLastError());
+  DG_CUDA_TRY(launch_plain(moe_gather_kernel, blocks, 256, st, static_cast<const uint8_t*>(q),
+                           reinterpret_cast<const uint32_t*>(sfa), T, K, kp, static_cast<const int32_t*>(src_of),
+                           M_cap, static_cast<uint8_t*>(a_perm), reinterpret_cast<uint32_t*>(sfa_perm)));
   return DG_OK;
 }
 
@@ -700,9 +742,9 @@ int dg_moe_unpermute_combine(const void* d_perm, const int32_t* row_of, const fl
   int r = device_info(&di);
   if (r) return r;
   const long long blocks = std::min<long long>((work + 255) / 256, 16LL * di.sms);
-  moe_combine_kernel<<<static_cast<int>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(d_perm), row_of, weights, T, topk, N, static_cast<__nv_bfloat16*>(out));
-  DG_CUDA_TRY(cudaGetLastError());
+  DG_CUDA_TRY(launch_plain(moe_combine_kernel, blocks, 256, static_cast<cudaStream_t>(stream),
+                           static_cast<const __nv_bfloat16*>(d_perm), row_of, weights, T, topk, N,
+                           static_cast<__nv_bfloat16*>(out)));
   return DG_OK;
 }
 

@@ -45,6 +45,11 @@
 // between atoms along K, LBO = 16 KB between 128-wide atoms along M/N.
 // Each CTA's share of an MN-major B tile is a whole number of 128 columns.
 //
+// SPLITK (with PIPES = 2): both pipelines work on every tile, pipeline p on
+// its half of the K groups, into its own accumulator; the epilogue adds the
+// two.  For problems of a few rows (decode) whose K loop is bound by the
+// issuing thread, this halves the loop without any workspace.
+//
 // PIPES = 2: every tcgen05 instruction costs its issuing thread
 // a fixed ~60-70 cycles, so one thread issuing the 4 MMAs + commit of a
 // 128x224x128 K block spends ~300 of the block's 448 tensor-pipe cycles on
@@ -237,12 +242,14 @@ __device__ __forceinline__ int contig_expert(const Tile& tl, const GemmArgs& p) 
   return e;
 }
 
-template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0>
+template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0,
+          bool SPLITK = false>
 __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
   using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>;
   static_assert(LAYOUT == 0 || MODE == MODE_DENSE, "MN-major operands are built for the dense GEMM only");
+  static_assert(!SPLITK || PIPES == 2, "split-K runs on two pipelines");
   constexpr bool kAmn = (LAYOUT & 1) != 0;
   constexpr bool kBmn = (LAYOUT & 2) != 0;
   constexpr bool kPair = CTAS == 2;
@@ -274,8 +281,14 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   const int sbase = pipe * L::kStagesPer;
   const int rbase = pipe * L::kSfRing;
   // With two pipelines, the i-th tile this CTA computes (skipped tiles not
-  // counted) belongs to pipeline i & 1.
-  auto take = [&](uint32_t& li) { return PIPES == 1 || static_cast<int>(li++ & 1) == pipe; };
+  // counted) belongs to pipeline i & 1; with split-K every tile belongs to both.
+  auto take = [&](uint32_t& li) { return PIPES == 1 || SPLITK || static_cast<int>(li++ & 1) == pipe; };
+  // K range of this pipeline, in groups of 4 K blocks (split-K: first or second half)
+  const int g_begin = SPLITK ? pipe * ((p.kp + 1) / 2) : 0;
+  const int g_end = SPLITK ? (pipe == 0 ? (p.kp + 1) / 2 : p.kp) : p.kp;
+  const int kb_begin = 4 * g_begin;
+  const int kb_end = min(num_kb, 4 * g_end);
+  const bool split_active = SPLITK && p.kp >= 2;  // otherwise the second accumulator stays unused
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -302,6 +315,10 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     tmem_alloc<CTAS>(tmem_holder, L::kTmemCols);
     tmem_relinquish<CTAS>();
   }
+  // Everything above touches no global memory, so it overlaps the previous
+  // grid's tail; from here on its results are visible.
+  grid_dep_wait();
+  grid_dep_launch();
   if (MODE == MODE_MASKED && warp == 2) {
     // counts[g] = clamp(masked_m[g], 0, M_max); prefix = running sum of tiles
     int run = 0;
@@ -353,7 +370,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       if (!take(li)) continue;
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
-      for (int kb = 0; kb < num_kb; ++kb, ++it) {
+      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
         const int s = sbase + static_cast<int>(it % L::kStagesPer);
         ok = wait_phase<false>(&empty_bar[s], ((it / L::kStagesPer) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
@@ -439,7 +456,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
         uint32_t accumulate = 0;
-        for (int kb0 = 0; kb0 < num_kb && ok; kb0 += 4, ++sf_group) {
+        for (int kb0 = kb_begin; kb0 < kb_end && ok; kb0 += 4, ++sf_group) {
           const uint32_t ring = sf_group % L::kSfRing;
           const uint32_t sf_col = sf_slot0 + (sf_group & 1) * L::kSfSlotCols;
           // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
@@ -462,7 +479,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
               tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8, (static_cast<uint64_t>(sfx_hi) << 32) |
                                                            (lo + (L::kSftMainBytes >> 4)));
           }
-          const int nk = min(4, num_kb - kb0);
+          const int nk = min(4, kb_end - kb0);
           uint32_t id = idesc0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -518,7 +535,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       if (!take(li)) continue;
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
-      for (int kp = 0; kp < p.kp; ++kp, ++group) {
+      for (int kp = g_begin; kp < g_end; ++kp, ++group) {
         const uint32_t ring = group % L::kSfRing;
         ok = wait_phase<false>(&sf_empty[rbase + ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
@@ -590,10 +607,11 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         expert = contig_expert<CTAS>(tl, p);
         if (expert < 0) continue;
       }
-      const uint32_t acc = local_tile % L::kNumAcc;
-      const uint32_t acc_use = local_tile / L::kNumAcc;
+      const uint32_t acc = SPLITK ? 0 : local_tile % L::kNumAcc;
+      const uint32_t acc_use = SPLITK ? local_tile : local_tile / L::kNumAcc;
       ++local_tile;
       bool ok = wait_phase<false>(&tmem_full[acc], acc_use & 1, abort_flag);
+      if (SPLITK && ok) ok = wait_phase<false>(&tmem_full[1], acc_use & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -699,7 +717,24 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         }
       };
 
-      if (any_valid) {
+      if (SPLITK && any_valid) {
+        // sum of the two pipelines' accumulators, chunk by chunk
+        uint32_t r[2][32];
+#pragma unroll 1
+        for (int i = 0; i < nmine; ++i) {
+          const int c = half + 2 * i;
+          const int col0 = n0 + 32 * c;
+          if (col0 >= p.N) break;
+          tmem_ld_32x32b_x32(t_row + 32 * c, r[0]);
+          if (split_active) tmem_ld_32x32b_x32(t_row + L::kAccStride + 32 * c, r[1]);
+          tmem_wait_ld();
+          if (split_active) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) r[0][j] = __float_as_uint(__uint_as_float(r[0][j]) + __uint_as_float(r[1][j]));
+          }
+          store_chunk(r[0], col0);
+        }
+      } else if (any_valid) {
         uint32_t r[2][32];
         if (nmine > 0 && n0 + 32 * half < p.N) tmem_ld_32x32b_x32(t_row + 32 * half, r[0]);
         tmem_wait_ld();
@@ -718,6 +753,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       if (lane == 0) {
         if constexpr (kPair) mbar_arrive_remote(empty0 + 8 * acc);
         else mbar_arrive(&tmem_empty[acc]);
+        if constexpr (SPLITK) mbar_arrive(&tmem_empty[1]);
       }
     }
     if (lane == 0) bulk_wait_group<0>();

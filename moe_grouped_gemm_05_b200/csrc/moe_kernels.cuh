@@ -16,6 +16,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace dg {
 
 constexpr int kMoeMaxExperts = 1024;
@@ -28,6 +30,8 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
   __shared__ int cnt[kMoeMaxExperts];
   __shared__ int warp_tot[32];
   __shared__ int seg_off, total_rows, running;
+  grid_dep_wait();
+  grid_dep_launch();
   const int e = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < G; i += blockDim.x) cnt[i] = 0;
@@ -104,6 +108,8 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
                                                         int T, int K, int kp, const int32_t* __restrict__ src_of,
                                                         int M_cap, uint8_t* __restrict__ a_perm,
                                                         uint32_t* __restrict__ sfa_perm) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int chunks = K / 16;
   const int t4 = (T + 3) & ~3;
   const long long total = static_cast<long long>(M_cap) * chunks;
@@ -123,6 +129,8 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
 __global__ void __launch_bounds__(256) moe_combine_kernel(const __nv_bfloat16* __restrict__ d, const int32_t* __restrict__ row_of,
                                                          const float* __restrict__ w, int T, int topk, int N,
                                                          __nv_bfloat16* __restrict__ out) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int chunks = N / 8;
   const long long total = static_cast<long long>(T) * chunks;
   for (long long u = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u < total;

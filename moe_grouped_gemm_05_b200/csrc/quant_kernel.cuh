@@ -14,6 +14,8 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "ptx.cuh"
+
 namespace dg {
 
 __device__ __forceinline__ float load_as_float(const __nv_bfloat16* p, int i) { return __bfloat162float(p[i]); }
@@ -78,6 +80,8 @@ template <typename T>
 __global__ void __launch_bounds__(256) quantize_1x128_kernel(const T* __restrict__ x, uint8_t* __restrict__ q,
                                                             uint32_t* __restrict__ sf, int batch, int M, int K,
                                                             int kp, int mn4) {
+  grid_dep_wait();
+  grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   const long long units = static_cast<long long>(batch) * mn4 * kp;

@@ -14,9 +14,11 @@ from helpers import bits, check_close, packed, to_device
 pytestmark = pytest.mark.gpu
 
 # (block_n, ctas, pipes)
-BUILT = [(128, 1, 1), (224, 1, 1), (256, 1, 1), (128, 2, 1), (224, 2, 1), (256, 2, 1), (224, 2, 2), (128, 2, 2)]
-BUILT_1CTA = [c for c in BUILT if c[1] == 1]
-BUILT_CONTIG = BUILT_1CTA + [(224, 2, 2)]  # the contiguous layout's configurations
+# (64|128, 1, 2) are the split-K tiles: both pipelines on every tile, each on half of K
+BUILT = [(128, 1, 1), (224, 1, 1), (256, 1, 1), (128, 2, 1), (224, 2, 1), (256, 2, 1), (224, 2, 2), (128, 2, 2),
+         (64, 1, 1), (64, 1, 2), (128, 1, 2)]
+BUILT_1CTA = [c for c in BUILT if c[1] == 1 and c[2] == 1]
+BUILT_CONTIG = [(128, 1, 1), (224, 1, 1), (256, 1, 1), (224, 2, 2)]  # the contiguous layout's configurations
 SENTINEL = 0xDEAD
 
 
