@@ -4,7 +4,9 @@
 One step = one pass of the whole hot path over one batch of synthetic input:
 pack the activation scales (fp32 power-of-two -> UE8M0 int32, the packing
 kernel) and run the GEMM (TMA ring -> block-scaled tcgen05 MMA -> epilogue)
-on them.  Weight scales are packed once, as a deployment would.
+on them (--fused-pack: the GEMM reads the fp32 scales and its scale-producer
+warp packs them, one launch per step).  Weight scales are packed once, as a
+deployment would.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
@@ -48,6 +50,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end loop (0 = min(steps, 100))")
     ap.add_argument("--eager", action="store_true", help="time host-issued launches instead of a CUDA graph")
+    ap.add_argument("--fused-pack", action="store_true",
+                    help="let the GEMM read A's fp32 scales and pack them itself instead of a packing launch")
     return ap.parse_args()
 
 
@@ -205,12 +209,14 @@ def make_device_sets(p, dg, torch, dev):
     return sets, per_set
 
 
-def gemm_call(p, dg, s):
+def gemm_call(p, dg, s, fp32_sfa=False):
+    """The GEMM of a step; with fp32_sfa it reads A's fp32 scales and packs them itself."""
+    sfa = s["sfa32"] if fp32_sfa else s["sfa"]
     if p.kind == "dense":
-        return dg.fp8_gemm_nt(s["a"], s["sfa"], s["b"], s["sfb"], s["d"])
+        return dg.fp8_gemm_nt(s["a"], sfa, s["b"], s["sfb"], s["d"])
     if p.kind == "contiguous":
-        return dg.m_grouped_fp8_gemm_nt_contiguous(s["a"], s["sfa"], s["b"], s["sfb"], s["m_indices"], s["d"])
-    return dg.m_grouped_fp8_gemm_nt_masked(s["a"], s["sfa"], s["b"], s["sfb"], s["masked_m"], s["d"])
+        return dg.m_grouped_fp8_gemm_nt_contiguous(s["a"], sfa, s["b"], s["sfb"], s["m_indices"], s["d"])
+    return dg.m_grouped_fp8_gemm_nt_masked(s["a"], sfa, s["b"], s["sfb"], s["masked_m"], s["d"])
 
 
 def pack_call(dg, lib, s, torch):
@@ -347,10 +353,13 @@ def run_ours(args):
     nsets = len(sets)
     stream = torch.cuda.current_stream()
 
+    fused = args.fused_pack
+
     def step(i):
         s = sets[i % nsets]
-        pack_call(dg, lib, s, torch)
-        gemm_call(p, dg, s)
+        if not fused:
+            pack_call(dg, lib, s, torch)
+        gemm_call(p, dg, s, fp32_sfa=fused)
 
     for i in range(args.warmup):
         step(i)
@@ -374,7 +383,7 @@ def run_ours(args):
             gemm_graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gemm_graph, stream=cap):
                 for i in range(args.steps):
-                    gemm_call(p, dg, sets[i % nsets])
+                    gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
         torch.cuda.synchronize()
         step_graph.replay()  # upload + untimed pass
         gemm_graph.replay()
@@ -403,7 +412,7 @@ def run_ours(args):
         gemm_graph.replay()
     else:
         for i in range(args.steps):
-            gemm_call(p, dg, sets[i % nsets])
+            gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
     g1.record(stream)
     torch.cuda.synchronize()
     sampler.stop()
@@ -423,8 +432,9 @@ def run_ours(args):
     for _ in range(2):
         s0["a"].view(torch.uint8).copy_(a_host, non_blocking=True)
         s0["sfa32"].copy_(sfa_host, non_blocking=True)
-        pack_call(dg, lib, s0, torch)
-        gemm_call(p, dg, s0)
+        if not fused:
+            pack_call(dg, lib, s0, torch)
+        gemm_call(p, dg, s0, fp32_sfa=fused)
         d_host.copy_(s0["d"], non_blocking=True)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -434,8 +444,9 @@ def run_ours(args):
     for _ in range(e2e_steps):
         s0["a"].view(torch.uint8).copy_(a_host, non_blocking=True)
         s0["sfa32"].copy_(sfa_host, non_blocking=True)
-        pack_call(dg, lib, s0, torch)
-        gemm_call(p, dg, s0)
+        if not fused:
+            pack_call(dg, lib, s0, torch)
+        gemm_call(p, dg, s0, fp32_sfa=fused)
         d_host.copy_(s0["d"], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -468,7 +479,8 @@ def run_ours(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
         "config": {"workload": args.workload, "kind": p.kind, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
                    "valid_rows": p.valid_rows, "kernel_config": kernel_desc,
-                   "step": "pack activation scales (fp32 -> UE8M0 int32) + GEMM",
+                   "step": ("GEMM reading A's fp32 scales, packed to UE8M0 in its scale-producer warp"
+                            if fused else "pack activation scales (fp32 -> UE8M0 int32) + GEMM"),
                    "timing": "eager launches" if args.eager else "CUDA-graph replay of the K steps",
                    "l2": f"inputs rotate over {nsets} device copies ({nsets * per_set / 1e6:.0f} MB > 2x L2)"},
         "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
@@ -476,7 +488,7 @@ def run_ours(args):
                      "kernel": "fp8_gemm_kernel", "kernel_ms_avg": gemm_avg_ms},
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": e2e_steps},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 if fused else 2) * args.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "device_error": err,
     }

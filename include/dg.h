@@ -72,6 +72,26 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
                    int M, int N, int K, void* stream);
 
 /*
+ * The three GEMMs of the hot path with A's scales given as fp32 powers of two
+ * instead of packed words: sfa is float [M][K/128] (dense), [M_total][K/128]
+ * (contiguous) or [G][M_max][K/128] (masked), row-major, 4-byte aligned.  The
+ * kernel's scale-producer warp packs each group of four exponents as
+ * dg_pack_sf_ue8m0 would (the nightvoyager.top report, "SF 双 path": the
+ * library turns FP32 scales into the packed UE8M0 layout), so a step needs
+ * no separate packing launch.  A scale that is not a power of two in UE8M0
+ * range is used as 2^-127 and sets DG_DEVERR_BAD_SCALE.  Everything else
+ * (B's packed scales, layouts, errors) is as in the packed-word entry points.
+ */
+int dg_fp8_gemm_nt_fp32sfa(const void* a, const float* sfa, const void* b, const int32_t* sfb, void* d,
+                           int M, int N, int K, void* stream);
+int dg_m_grouped_fp8_gemm_nt_contiguous_fp32sfa(const void* a, const float* sfa, const void* b,
+                                                const int32_t* sfb, void* d, const int32_t* m_indices,
+                                                int M_total, int N, int K, int num_groups, void* stream);
+int dg_m_grouped_fp8_gemm_nt_masked_fp32sfa(const void* a, const float* sfa, const void* b,
+                                            const int32_t* sfb, void* d, const int32_t* masked_m,
+                                            int num_groups, int M_max, int N, int K, void* stream);
+
+/*
  * Dense FP8 GEMM with the other operand layouts (the ssnai.com analysis,
  * "SM90 vs SM100": SM100 serves NT, TN, NN and TT).  The first letter is the
  * LHS, the second the RHS; N = not transposed, T = transposed, so NT is

@@ -50,6 +50,9 @@ def load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     vp, i32p, i = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int
     lib.dg_fp8_gemm_nt.argtypes = [vp, i32p, vp, i32p, vp, i, i, i, vp]
+    lib.dg_fp8_gemm_nt_fp32sfa.argtypes = [vp, vp, vp, i32p, vp, i, i, i, vp]
+    lib.dg_m_grouped_fp8_gemm_nt_contiguous_fp32sfa.argtypes = [vp, vp, vp, i32p, vp, i32p, i, i, i, i, vp]
+    lib.dg_m_grouped_fp8_gemm_nt_masked_fp32sfa.argtypes = [vp, vp, vp, i32p, vp, i32p, i, i, i, i, vp]
     for name in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
         getattr(lib, name).argtypes = [vp, i32p, vp, i32p, vp, i, i, i, vp]
     lib.dg_m_grouped_fp8_gemm_nt_contiguous.argtypes = [vp, i32p, vp, i32p, vp, i32p, i, i, i, i, vp]
@@ -164,20 +167,37 @@ def quantize_fp8_1x128(x: torch.Tensor, q=None, sf=None):
     return q, sf
 
 
+def _sfa_kind(sfa: torch.Tensor, rows_shape: tuple, K: int) -> bool:
+    """True when sfa holds fp32 scales [..rows.., K/128] (packed in the kernel), False for packed int32 words."""
+    if sfa.dtype == torch.float32:
+        if not sfa.is_cuda or not sfa.is_contiguous() or tuple(sfa.shape) != (*rows_shape, K // 128):
+            raise ValueError(f"fp32 sfa must be a contiguous CUDA tensor of shape {(*rows_shape, K // 128)}")
+        return True
+    _i32(sfa, "sfa")
+    return False
+
+
 def fp8_gemm_nt(a, sfa, b, sfb, d=None) -> torch.Tensor:
-    """D[M,N] (bf16) = A[M,K] . B[N,K]^T with packed 1x128 / 128x128 UE8M0 scales."""
-    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb")
+    """D[M,N] (bf16) = A[M,K] . B[N,K]^T with 1x128 / 128x128 UE8M0 scales.
+
+    sfa: packed int32 words [ceil(Kb/4), align4(M)], or the fp32 power-of-two scales [M, Kb]
+    (then the GEMM packs them itself: no separate packing launch).
+    """
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfb, "sfb")
     M, K = a.shape
     N, Kb_ = b.shape
     if Kb_ != K:
         raise ValueError("a and b disagree on K")
-    if tuple(sfa.shape) != packed_sf_words(M, K // 128) or tuple(sfb.shape) != packed_sf_words(-(-N // 128), K // 128):
+    fp32_sfa = _sfa_kind(sfa, (M,), K)
+    if (not fp32_sfa and tuple(sfa.shape) != packed_sf_words(M, K // 128)) or \
+            tuple(sfb.shape) != packed_sf_words(-(-N // 128), K // 128):
         raise ValueError("packed scale shapes do not match [ceil(Kb/4), align4(MN)]")
     if d is None:
         d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
         raise ValueError("d must be a contiguous bf16 [M, N] tensor")
-    _check(load().dg_fp8_gemm_nt(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
+    fn = load().dg_fp8_gemm_nt_fp32sfa if fp32_sfa else load().dg_fp8_gemm_nt
+    _check(fn(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), M, N, K, _stream()))
     return d
 
 
@@ -229,34 +249,40 @@ def fp8_gemm_nt_ex(a, sfa, b, sfb, c=None, d=None, recipe_b: int = 128, out_dtyp
 
 
 def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices, d=None) -> torch.Tensor:
-    """Contiguous-layout grouped GEMM: D[m] = A[m] . B[m_indices[m]]^T; -1 rows untouched."""
-    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb"), _i32(m_indices, "m_indices")
+    """Contiguous-layout grouped GEMM: D[m] = A[m] . B[m_indices[m]]^T; -1 rows untouched.
+
+    sfa: packed words or fp32 scales [M_total, Kb] (packed in the kernel)."""
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfb, "sfb"), _i32(m_indices, "m_indices")
     M, K = a.shape
     G, N, Kb_ = b.shape
     if Kb_ != K or m_indices.shape != (M,):
         raise ValueError("shape mismatch")
+    fp32_sfa = _sfa_kind(sfa, (M,), K)
     if d is None:
         d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
         raise ValueError("d must be a contiguous bf16 [M_total, N] tensor")
-    _check(load().dg_m_grouped_fp8_gemm_nt_contiguous(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d),
-                                                       _ptr(m_indices), M, N, K, G, _stream()))
+    fn = load().dg_m_grouped_fp8_gemm_nt_contiguous_fp32sfa if fp32_sfa else load().dg_m_grouped_fp8_gemm_nt_contiguous
+    _check(fn(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(m_indices), M, N, K, G, _stream()))
     return d
 
 
 def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m, d=None) -> torch.Tensor:
-    """Masked-layout grouped GEMM: rows m < masked_m[g] of expert g; other rows untouched."""
-    _fp8(a, "a"), _fp8(b, "b"), _i32(sfa, "sfa"), _i32(sfb, "sfb"), _i32(masked_m, "masked_m")
+    """Masked-layout grouped GEMM: rows m < masked_m[g] of expert g; other rows untouched.
+
+    sfa: packed words or fp32 scales [G, M_max, Kb] (packed in the kernel)."""
+    _fp8(a, "a"), _fp8(b, "b"), _i32(sfb, "sfb"), _i32(masked_m, "masked_m")
     G, M_max, K = a.shape
     Gb, N, Kb_ = b.shape
     if Gb != G or Kb_ != K or masked_m.shape != (G,):
         raise ValueError("shape mismatch")
+    fp32_sfa = _sfa_kind(sfa, (G, M_max), K)
     if d is None:
         d = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (G, M_max, N) or not d.is_contiguous():
         raise ValueError("d must be a contiguous bf16 [G, M_max, N] tensor")
-    _check(load().dg_m_grouped_fp8_gemm_nt_masked(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d),
-                                                   _ptr(masked_m), G, M_max, N, K, _stream()))
+    fn = load().dg_m_grouped_fp8_gemm_nt_masked_fp32sfa if fp32_sfa else load().dg_m_grouped_fp8_gemm_nt_masked
+    _check(fn(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(d), _ptr(masked_m), G, M_max, N, K, _stream()))
     return d
 
 

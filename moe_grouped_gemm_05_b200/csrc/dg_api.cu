@@ -465,21 +465,27 @@ static int build_maps_cached(CUtensorMap* maps, const Config* cfg, const void* a
   return DG_OK;
 }
 
-static void fill_scale_args(GemmArgs* args, const int32_t* sfa, const int32_t* sfb, int rowsA, int N, int K,
-                            int sfb_gran = 128) {
+// sfa is either packed UE8M0 words or, with sfa_fp32, the fp32 scales [G][rowsA][K/128] that the
+// kernel's scale producer packs on the fly.
+static void fill_scale_args(GemmArgs* args, const void* sfa, const int32_t* sfb, int rowsA, int N, int K,
+                            int sfb_gran = 128, bool sfa_fp32 = false) {
   args->kp = (K / 128 + 3) / 4;
   args->mn4a = (rowsA + 3) / 4 * 4;
   args->sfb_gran = sfb_gran;
   args->nb4 = ((N + sfb_gran - 1) / sfb_gran + 3) / 4 * 4;
-  args->sfa = reinterpret_cast<const uint32_t*>(sfa);
+  args->sfa = sfa_fp32 ? nullptr : static_cast<const uint32_t*>(sfa);
+  args->sfa_f32 = sfa_fp32 ? static_cast<const float*>(sfa) : nullptr;
+  args->sfa_f32_vec = sfa_fp32 && (K / 128) % 4 == 0 && aligned16(sfa);
   args->sfb = reinterpret_cast<const uint32_t*>(sfb);
 }
 
-static int check_common(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb,
-                        void* d, int N, int K) {
+static int check_common(const void* a, const void* sfa, const void* b, const int32_t* sfb,
+                        void* d, int N, int K, bool sfa_fp32 = false) {
   if (!a || !sfa || !b || !sfb || !d) return fail(DG_ERR_NULL, "a, sfa, b, sfb and d must be non-NULL");
-  if (!aligned16(a) || !aligned16(b) || !aligned16(d) || !aligned16(sfa) || !aligned16(sfb))
-    return fail(DG_ERR_ALIGN, "a, sfa, b, sfb and d must be 16-byte aligned");
+  if (!aligned16(a) || !aligned16(b) || !aligned16(d) || !aligned16(sfb))
+    return fail(DG_ERR_ALIGN, "a, b, sfb and d must be 16-byte aligned");
+  if (sfa_fp32 ? (reinterpret_cast<uintptr_t>(sfa) & 3) != 0 : !aligned16(sfa))
+    return fail(DG_ERR_ALIGN, sfa_fp32 ? "fp32 sfa must be 4-byte aligned" : "sfa must be 16-byte aligned");
   if (K <= 0 || K % 128 != 0) return fail(DG_ERR_SHAPE, "K=%d must be a positive multiple of 128", K);
   if (N <= 0 || N % 16 != 0) return fail(DG_ERR_SHAPE, "N=%d must be a positive multiple of 16", N);
   return DG_OK;
@@ -515,18 +521,7 @@ __global__ void pack_sf_ue8m0_kernel(const float* __restrict__ sf, uint32_t* __r
       for (int j = 0; j < 4; ++j) {
         const int k = 4 * p + j;
         if (k >= kb) break;
-        const uint32_t bits = __float_as_uint(sf[(static_cast<long long>(bt) * mn + m) * kb + k]);
-        const uint32_t expf = (bits >> 23) & 0xFFu;
-        const uint32_t mant = bits & 0x7FFFFFu;
-        uint32_t byte = 0;
-        if ((bits >> 31) == 0 && expf >= 1 && expf <= 254 && mant == 0) {
-          byte = expf;
-        } else if (bits == 0x00400000u) {  // 2^-127, the fp32 subnormal of UE8M0 byte 0
-          byte = 0;
-        } else {
-          bad = true;
-        }
-        word |= byte << (8 * j);
+        word |= ue8m0_byte_checked(__float_as_uint(sf[(static_cast<long long>(bt) * mn + m) * kb + k]), bad) << (8 * j);
       }
     }
     out[i] = word;
@@ -541,9 +536,9 @@ using namespace dg;
 // ==================================================================== C ABI
 
 template <int HMODE>
-static int gemm_dense(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d, int M,
-                      int N, int K, void* stream) {
-  int r = check_common(a, sfa, b, sfb, d, N, K);
+static int gemm_dense(const void* a, const void* sfa, const void* b, const int32_t* sfb, void* d, int M,
+                      int N, int K, void* stream, bool sfa_fp32 = false) {
+  int r = check_common(a, sfa, b, sfb, d, N, K, sfa_fp32);
   if (r) return r;
   if (M < 0) return fail(DG_ERR_SHAPE, "M=%d must be >= 0", M);
   if (M == 0) return DG_OK;
@@ -565,7 +560,7 @@ static int gemm_dense(const void* a, const int32_t* sfa, const void* b, const in
   args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
   args.raster_m = raster_group(args.num_m_blocks);
   args.d = static_cast<__nv_bfloat16*>(d);
-  fill_scale_args(&args, sfa, sfb, M, N, K);
+  fill_scale_args(&args, sfa, sfb, M, N, K, 128, sfa_fp32);
   const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
   return launch<HMODE>(cfg, grid_size(di.sms, tiles, cfg), maps, args, static_cast<cudaStream_t>(stream));
 }
@@ -753,6 +748,11 @@ int dg_fp8_gemm_nt(const void* a, const int32_t* sfa, const void* b, const int32
   return gemm_dense<MODE_DENSE>(a, sfa, b, sfb, d, M, N, K, stream);
 }
 
+int dg_fp8_gemm_nt_fp32sfa(const void* a, const float* sfa, const void* b, const int32_t* sfb, void* d,
+                           int M, int N, int K, void* stream) {
+  return gemm_dense<MODE_DENSE>(a, sfa, b, sfb, d, M, N, K, stream, true);
+}
+
 int dg_fp8_gemm_nn(const void* a, const int32_t* sfa, const void* b, const int32_t* sfb, void* d,
                    int M, int N, int K, void* stream) {
   return gemm_dense<MODE_DENSE_MN + 1>(a, sfa, b, sfb, d, M, N, K, stream);
@@ -804,10 +804,10 @@ int dg_fp8_gemm_nt_ex(const void* a, const int32_t* sfa, const void* b, const in
   return launch<MODE_DENSE>(cfg, grid_size(di.sms, tiles, cfg), maps, args, static_cast<cudaStream_t>(stream));
 }
 
-int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
-                                        const int32_t* sfb, void* d, const int32_t* m_indices,
-                                        int M_total, int N, int K, int num_groups, void* stream) {
-  int r = check_common(a, sfa, b, sfb, d, N, K);
+static int contiguous_impl(const void* a, const void* sfa, const void* b, const int32_t* sfb, void* d,
+                           const int32_t* m_indices, int M_total, int N, int K, int num_groups, void* stream,
+                           bool sfa_fp32) {
+  int r = check_common(a, sfa, b, sfb, d, N, K, sfa_fp32);
   if (r) return r;
   if (!m_indices) return fail(DG_ERR_NULL, "m_indices must be non-NULL");
   if (num_groups <= 0) return fail(DG_ERR_SHAPE, "num_groups=%d must be positive", num_groups);
@@ -830,16 +830,28 @@ int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const
   args.raster_m = raster_group(args.num_m_blocks);
   args.m_indices = m_indices;
   args.d = static_cast<__nv_bfloat16*>(d);
-  fill_scale_args(&args, sfa, sfb, M_total, N, K);
+  fill_scale_args(&args, sfa, sfb, M_total, N, K, 128, sfa_fp32);
   const long long tiles = static_cast<long long>(args.num_m_blocks) * args.num_n_blocks;
   return launch<MODE_CONTIG>(cfg, grid_size(di.sms, tiles, cfg), maps, args,
                              static_cast<cudaStream_t>(stream));
 }
 
-int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
-                                    const int32_t* sfb, void* d, const int32_t* masked_m,
-                                    int num_groups, int M_max, int N, int K, void* stream) {
-  int r = check_common(a, sfa, b, sfb, d, N, K);
+int dg_m_grouped_fp8_gemm_nt_contiguous(const void* a, const int32_t* sfa, const void* b,
+                                        const int32_t* sfb, void* d, const int32_t* m_indices,
+                                        int M_total, int N, int K, int num_groups, void* stream) {
+  return contiguous_impl(a, sfa, b, sfb, d, m_indices, M_total, N, K, num_groups, stream, false);
+}
+
+int dg_m_grouped_fp8_gemm_nt_contiguous_fp32sfa(const void* a, const float* sfa, const void* b,
+                                                const int32_t* sfb, void* d, const int32_t* m_indices,
+                                                int M_total, int N, int K, int num_groups, void* stream) {
+  return contiguous_impl(a, sfa, b, sfb, d, m_indices, M_total, N, K, num_groups, stream, true);
+}
+
+static int masked_impl(const void* a, const void* sfa, const void* b, const int32_t* sfb, void* d,
+                       const int32_t* masked_m, int num_groups, int M_max, int N, int K, void* stream,
+                       bool sfa_fp32) {
+  int r = check_common(a, sfa, b, sfb, d, N, K, sfa_fp32);
   if (r) return r;
   if (!masked_m) return fail(DG_ERR_NULL, "masked_m must be non-NULL");
   if (num_groups <= 0 || num_groups > kMaxMaskedGroups)
@@ -865,10 +877,22 @@ int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const voi
   args.raster_m = 1;
   args.masked_m = masked_m;
   args.d = static_cast<__nv_bfloat16*>(d);
-  fill_scale_args(&args, sfa, sfb, M_max, N, K);
+  fill_scale_args(&args, sfa, sfb, M_max, N, K, 128, sfa_fp32);
   const long long max_tiles = static_cast<long long>(num_groups) * args.num_m_blocks * args.num_n_blocks;
   return launch<MODE_MASKED>(cfg, grid_size(di.sms, max_tiles, cfg), maps, args,
                              static_cast<cudaStream_t>(stream));
+}
+
+int dg_m_grouped_fp8_gemm_nt_masked(const void* a, const int32_t* sfa, const void* b,
+                                    const int32_t* sfb, void* d, const int32_t* masked_m,
+                                    int num_groups, int M_max, int N, int K, void* stream) {
+  return masked_impl(a, sfa, b, sfb, d, masked_m, num_groups, M_max, N, K, stream, false);
+}
+
+int dg_m_grouped_fp8_gemm_nt_masked_fp32sfa(const void* a, const float* sfa, const void* b,
+                                            const int32_t* sfb, void* d, const int32_t* masked_m,
+                                            int num_groups, int M_max, int N, int K, void* stream) {
+  return masked_impl(a, sfa, b, sfb, d, masked_m, num_groups, M_max, N, K, stream, true);
 }
 
 }  // extern "C"

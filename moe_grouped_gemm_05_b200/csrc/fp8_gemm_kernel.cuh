@@ -20,20 +20,26 @@
 // fetches half of the B tile it would need alone.  No load is multicast.
 //
 // Roles (one CTA per SM, persistent over output tiles):
-//   warp 0     producer: TMA loads of A/B K-blocks into a STAGES-deep ring.
-//   warp 1     TMEM owner; in the first CTA of a pair also the MMA issuer:
-//              tcgen05.cp of the scales, tcgen05.mma, commits of stage
-//              releases and finished accumulators (to both CTAs of a pair).
-//   warps 2-5 and the last four warps of the block
-//              epilogue: tcgen05.ld of this CTA's accumulator rows (two warps
-//              per TMEM lane quarter, alternate 32-column chunks), BF16 RNE,
-//              swizzled staging + TMA store for fully valid 32-row slices,
-//              predicated stores for slices holding padding/masked rows.
-//   warp 6     scale producer: for every group of 4 K-blocks, the packed UE8M0
-//              words of the tile, rearranged into the tensor-memory scale
-//              layout (row/column j of a 128-group at lane j%32, column j/32),
-//              into a 2- or 4-deep ring of its own, so the load latency of
-//              the words never sits on the TMA issue path.
+//   MMA issuer   TMEM owner (warp 0); in the first CTA of a pair the issuer:
+//                tcgen05.cp of the scales, tcgen05.mma, commits of stage
+//                releases and finished accumulators (to both CTAs of a pair).
+//   producer     TMA loads of A/B K-blocks into a STAGES-deep ring.
+//   scale        for every group of 4 K-blocks, the packed UE8M0 words of
+//   producer     the tile (or fp32 scales packed here), rearranged into the
+//                tensor-memory scale layout (row/column j of a 128-group at
+//                lane j%32, column j/32), into a 2- or 4-deep ring of its own,
+//                so the load latency of the words never sits on the TMA path.
+//   epilogue     eight warps: tcgen05.ld of this CTA's accumulator rows (two
+//                warps per TMEM lane quarter, alternate 32-column chunks),
+//                BF16 RNE, swizzled staging + TMA store for fully valid 32-row
+//                slices, predicated stores for slices with padding/masked rows.
+// Warp w runs on sub-partition w % 4, which also fixes the TMEM lane quarter
+// it may read.  The issuing threads are sensitive to other warps' instructions
+// on their sub-partition, so they share theirs only with a (light) producer
+// and two epilogue warps; the scale producers sit on the other two:
+//   PIPES = 1: warp 0 issuer, 1 producer, 2 scale producer, 3-10 epilogue.
+//   PIPES = 2: warps 0/1 issuers, 2/3 scale producers, 4/5 producers (of
+//              pipelines 0/1), 6-13 epilogue.
 // Accumulators are double-buffered in TMEM when they fit, so the epilogue of
 // tile i overlaps the MMAs of tile i+1.
 //
@@ -55,8 +61,8 @@
 // 128x224x128 K block spends ~300 of the block's 448 tensor-pipe cycles on
 // issue alone and, with its waits, cannot keep the pipe busy.  The cost is
 // per thread: two threads issuing into two accumulators overlap.  So the CTA
-// runs two copies of the load/issue/scale pipeline (warps 0, 1, 6 and 7, 8,
-// 9), each with half of the stage ring, its own scale ring and scale slots
+// runs two copies of the load/issue/scale pipeline (warps 0, 4, 2 and 1, 5,
+// 3), each with half of the stage ring, its own scale ring and scale slots
 // in TMEM, taking alternate tiles of the CTA: tile i goes to pipeline i & 1
 // and accumulator i & 1.  The epilogue warps drain the accumulators in tile
 // order, as with one pipeline.
@@ -74,10 +80,9 @@ __device__ int g_dg_error = 0;
 enum : int { MODE_DENSE = 0, MODE_CONTIG = 1, MODE_MASKED = 2 };
 
 constexpr int kBK = 128;
-// warps 0, 1, 6: producer, MMA issuer, scale producer; 2-5 and the last four:
-// epilogue; PIPES = 2 adds a second producer, issuer and scale warp (7, 8, 9)
+// per pipeline an MMA issuer, a producer and a scale producer; eight epilogue warps
 template <int PIPES>
-constexpr int kThreadsFor = 32 * (11 + 3 * (PIPES - 1));
+constexpr int kThreadsFor = 32 * (8 + 3 * PIPES);
 constexpr int kThreads = kThreadsFor<1>;
 constexpr int kMaxMaskedGroups = 512;
 constexpr int kMaxSmem = 232448;                  // opt-in shared memory per block on sm_100
@@ -93,7 +98,9 @@ struct GemmArgs {
   int mn4a;           // words of packed A scales along M: align4(rows)
   int nb4;            // words of packed B scales along N: align4(ceil(N / sfb_gran))
   int sfb_gran;       // rows of B per scale: 128 (128x128 blocks) or 1 (1x128 per row)
-  const uint32_t* sfa;
+  const uint32_t* sfa;     // packed UE8M0 words of A, or nullptr when sfa_f32 is given
+  const float* sfa_f32;    // A's fp32 power-of-two scales [G][rows][K/128], packed by the scale producer
+  int sfa_f32_vec;         // 1: rows of sfa_f32 are 16-byte aligned (K/128 % 4 == 0): one 16-byte load per word
   const uint32_t* sfb;
   const int32_t* m_indices;
   const int32_t* masked_m;
@@ -151,6 +158,35 @@ struct Layout {
 struct Tile {
   int m_blk, n_blk, g;
 };
+
+// UE8M0 byte of an fp32 scale: the exponent field of a positive normal power
+// of two, 0 for 2^-127 (the fp32 subnormal 0x00400000); anything else is not
+// representable and gives byte 0 with `bad` set.
+__device__ __forceinline__ uint32_t ue8m0_byte_checked(uint32_t bits, bool& bad) {
+  const uint32_t e = (bits >> 23) & 0xFFu;
+  if ((bits >> 31) == 0 && e >= 1 && e <= 254 && (bits & 0x7FFFFFu) == 0) return e;
+  if (bits != 0x00400000u) bad = true;
+  return 0u;
+}
+
+// Packed word of K blocks 4kp..4kp+3 of one row of fp32 scales (kbn blocks per row).
+__device__ __forceinline__ uint32_t pack_scale_word(const float* row, int kp, int kbn, bool vec) {
+  uint32_t word = 0;
+  bool bad = false;
+  if (vec) {  // 4 | kbn and 16-byte aligned rows: the word's four scales in one load
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(row) + kp);
+    word = ue8m0_byte_checked(v.x, bad) | (ue8m0_byte_checked(v.y, bad) << 8) |
+           (ue8m0_byte_checked(v.z, bad) << 16) | (ue8m0_byte_checked(v.w, bad) << 24);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = 4 * kp + j;
+      if (k < kbn) word |= ue8m0_byte_checked(__float_as_uint(__ldg(row + k)), bad) << (8 * j);
+    }
+  }
+  if (bad) atomicOr(&g_dg_error, 0x1);
+  return word;
+}
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting
 // (another role gave up) or this wait exceeded its limit (sets the error word).
@@ -275,9 +311,12 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   const uint32_t rank = kPair ? cluster_cta_rank() : 0;
   const int unit0 = kPair ? static_cast<int>(blockIdx.x / 2) : static_cast<int>(blockIdx.x);
   const int units = kPair ? static_cast<int>(gridDim.x / 2) : static_cast<int>(gridDim.x);
-  // pipeline of this warp (warps 7, 8, 9 mirror warps 0, 1, 6) and its share of the rings
-  constexpr int kEpiWarp2 = PIPES == 2 ? 10 : 7;  // first warp of the second epilogue set
-  const int pipe = (PIPES == 2 && warp >= 7 && warp < kEpiWarp2) ? 1 : 0;
+  // role and pipeline of this warp, and the pipeline's share of the rings
+  constexpr int kEpi0 = 3 * PIPES;  // first epilogue warp
+  const bool is_issuer = warp < PIPES;
+  const bool is_producer = PIPES == 2 ? (warp == 4 || warp == 5) : warp == 1;
+  const bool is_scale = PIPES == 2 ? (warp == 2 || warp == 3) : warp == 2;
+  const int pipe = (PIPES == 2 && warp < kEpi0) ? (warp & 1) : 0;
   const int sbase = pipe * L::kStagesPer;
   const int rbase = pipe * L::kSfRing;
   // With two pipelines, the i-th tile this CTA computes (skipped tiles not
@@ -311,7 +350,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     prefetch_tensormap(&tm_b);
     prefetch_tensormap(&tm_d);
   }
-  if (warp == 1) {
+  __syncwarp();
+  if (warp == 0) {
     tmem_alloc<CTAS>(tmem_holder, L::kTmemCols);
     tmem_relinquish<CTAS>();
   }
@@ -319,7 +359,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   // grid's tail; from here on its results are visible.
   grid_dep_wait();
   grid_dep_launch();
-  if (MODE == MODE_MASKED && warp == 2) {
+  if (MODE == MODE_MASKED && warp == kEpi0) {
     // counts[g] = clamp(masked_m[g], 0, M_max); prefix = running sum of tiles
     int run = 0;
     for (int base = 0; base < p.G; base += 32) {
@@ -351,7 +391,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   const uint32_t tmem_base = *tmem_holder;
   const int ntiles = total_tiles<MODE, CTAS>(p, prefix);
 
-  if (warp == 0 || (PIPES == 2 && warp == 7)) {
+  if (is_producer) {
     // ============================================================ producer
     // Barrier of stage s in the MMA-issuing CTA, as a shared::cluster address.
     const uint32_t full0 = kPair ? mapa_shared(smem_u32(full_bar), 0) : smem_u32(full_bar);
@@ -409,7 +449,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         wait_phase_drain(&full_bar[sbase + i % L::kStagesPer], (i / L::kStagesPer) & 1);
     }
     __syncwarp();
-  } else if (warp == 1 || (PIPES == 2 && warp == 8)) {
+  } else if (is_issuer) {
     // ============================================================ MMA issuer
     // A single thread issues.  Each tcgen05 instruction costs the issuing
     // thread ~60 cycles and every other instruction a few more, against 448
@@ -517,7 +557,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       wait_phase_drain(&final_bar[pipe], 0);
     }
     __syncwarp();
-  } else if (warp == 6 || (PIPES == 2 && warp == 9)) {
+  } else if (is_scale) {
     // ============================================================ scale producer
     const uint32_t sf_full0 = kPair ? mapa_shared(smem_u32(sf_full + rbase), 0) : smem_u32(sf_full + rbase);
     uint32_t group = 0, li = 0;
@@ -541,12 +581,22 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         // lane r gathers rows / columns r, r+32, r+64, r+96 of each 128-group
-        const uint32_t* sfa_row = p.sfa + (static_cast<size_t>(grp_a) * p.kp + kp) * p.mn4a;
         uint32_t wa[4];
+        if (p.sfa_f32 != nullptr) {  // fp32 scales: pack this group's word here (the packing step, fused)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int m = m_base + 32 * i + lane;
-          wa[i] = m < p.mn4a ? __ldg(sfa_row + m) : 0u;
+          for (int i = 0; i < 4; ++i) {
+            const int m = m_base + 32 * i + lane;
+            wa[i] = m < p.rows ? pack_scale_word(p.sfa_f32 + (static_cast<size_t>(grp_a) * p.rows + m) * num_kb, kp,
+                                                 num_kb, p.sfa_f32_vec != 0)
+                               : 0u;
+          }
+        } else {
+          const uint32_t* sfa_row = p.sfa + (static_cast<size_t>(grp_a) * p.kp + kp) * p.mn4a;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int m = m_base + 32 * i + lane;
+            wa[i] = m < p.mn4a ? __ldg(sfa_row + m) : 0u;
+          }
         }
         const uint32_t* sfb_row = p.sfb + (static_cast<size_t>(grp_b) * p.kp + kp) * p.nb4;
         uint32_t wb[L::kNB128][4];
@@ -587,8 +637,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     // odd ones.  The tcgen05.ld of a warp's next chunk is in flight while the
     // current one is converted and stored.
     const int q = warp % 4;  // TMEM lane quarter this warp may access
-    const int half = warp >= kEpiWarp2 ? 1 : 0;
-    const int epi_idx = half ? 4 + (warp - kEpiWarp2) : warp - 2;
+    const int epi_idx = warp - kEpi0;
+    const int half = epi_idx >> 2;
     uint8_t* buf = smem + L::kOffEpi + epi_idx * L::kEpiBuf;  // staging for one TMA store
     const uint32_t empty0 = kPair ? mapa_shared(smem_u32(tmem_empty), 0) : smem_u32(tmem_empty);
     constexpr int kChunks = BN / 32;
@@ -602,7 +652,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         // expert of this CTA's own 128-row block (a pair's blocks may differ)
         const int own_blk = CTAS * tl.m_blk + static_cast<int>(rank);
         own_e = own_blk < p.rows / 128 ? __ldg(&p.m_indices[own_blk * 128]) : -1;
-        if ((own_e < -1 || own_e >= p.G) && warp == 2 && lane == 0 && tl.n_blk == 0 && tl.g == 0)
+        if ((own_e < -1 || own_e >= p.G) && warp == kEpi0 && lane == 0 && tl.n_blk == 0 && tl.g == 0)
           atomicOr(&g_dg_error, 0x2);
         expert = contig_expert<CTAS>(tl, p);
         if (expert < 0) continue;
@@ -763,7 +813,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
   if constexpr (kPair) cluster_sync(); else __syncthreads();
-  if (warp == 1) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc<CTAS>(tmem_base, L::kTmemCols);
   }
