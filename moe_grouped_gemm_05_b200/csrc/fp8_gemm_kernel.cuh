@@ -54,7 +54,9 @@
 // SPLITK (with PIPES = 2): both pipelines work on every tile, pipeline p on
 // its half of the K groups, into its own accumulator; the epilogue adds the
 // two.  For problems of a few rows (decode) whose K loop is bound by the
-// issuing thread, this halves the loop without any workspace.
+// issuing thread, this halves the loop without any workspace.  Without
+// SPLITK, two pipelines split the same way only the last tile of a CTA with
+// an odd tile count (dense and masked), which would otherwise run alone.
 //
 // PIPES = 2: every tcgen05 instruction costs its issuing thread
 // a fixed ~60-70 cycles, so one thread issuing the 4 MMAs + commit of a
@@ -319,15 +321,11 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   const int pipe = (PIPES == 2 && warp < kEpi0) ? (warp & 1) : 0;
   const int sbase = pipe * L::kStagesPer;
   const int rbase = pipe * L::kSfRing;
-  // With two pipelines, the i-th tile this CTA computes (skipped tiles not
-  // counted) belongs to pipeline i & 1; with split-K every tile belongs to both.
-  auto take = [&](uint32_t& li) { return PIPES == 1 || SPLITK || static_cast<int>(li++ & 1) == pipe; };
-  // K range of this pipeline, in groups of 4 K blocks (split-K: first or second half)
-  const int g_begin = SPLITK ? pipe * ((p.kp + 1) / 2) : 0;
-  const int g_end = SPLITK ? (pipe == 0 ? (p.kp + 1) / 2 : p.kp) : p.kp;
-  const int kb_begin = 4 * g_begin;
-  const int kb_end = min(num_kb, 4 * g_end);
-  const bool split_active = SPLITK && p.kp >= 2;  // otherwise the second accumulator stays unused
+  // With two pipelines and no split-K, the last tile of an odd count is split
+  // over both pipelines, so the last round does not run on one issuing
+  // thread.  The contiguous layout's tile count depends on device data and
+  // keeps plain alternation.
+  constexpr bool kTailSplit = PIPES == 2 && !SPLITK && MODE != MODE_CONTIG;
 
   // ---------------------------------------------------------------- set-up
   if (threadIdx.x == 0) {
@@ -390,6 +388,29 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int ntiles = total_tiles<MODE, CTAS>(p, prefix);
+  // Tile i of this CTA (skipped tiles not counted) is either split over both
+  // pipelines, each on half of the K groups into its own accumulator, or owned
+  // by pipeline tile_pipe(i); every role derives the same plan.
+  const int n_mine = ntiles > unit0 ? (ntiles - unit0 + units - 1) / units : 0;
+  const int g_half = (p.kp + 1) / 2;
+  auto tile_split = [&](uint32_t i) {
+    return PIPES == 2 && p.kp >= 2 &&
+           (SPLITK || (kTailSplit && (n_mine & 1) != 0 && static_cast<int>(i) == n_mine - 1));
+  };
+  auto tile_pipe = [&](uint32_t i) { return SPLITK ? 0 : static_cast<int>(i & 1); };
+  // Whether this warp's pipeline works on the next tile (li advances), and its K groups [gb, ge).
+  auto plan = [&](uint32_t& li, int& gb, int& ge) {
+    const uint32_t i = li++;
+    gb = 0;
+    ge = p.kp;
+    if (PIPES == 1) return true;
+    if (tile_split(i)) {
+      gb = pipe == 0 ? 0 : g_half;
+      ge = pipe == 0 ? g_half : p.kp;
+      return true;
+    }
+    return tile_pipe(i) == pipe;
+  };
 
   if (is_producer) {
     // ============================================================ producer
@@ -407,10 +428,12 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       } else if (MODE == MODE_MASKED) {
         grp_a = grp_b = tl.g;
       }
-      if (!take(li)) continue;
+      int gb, ge;
+      if (!plan(li, gb, ge)) continue;
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
-      for (int kb = kb_begin; kb < kb_end; ++kb, ++it) {
+      const int kb_hi = min(num_kb, 4 * ge);
+      for (int kb = 4 * gb; kb < kb_hi; ++kb, ++it) {
         const int s = sbase + static_cast<int>(it % L::kStagesPer);
         ok = wait_phase<false>(&empty_bar[s], ((it / L::kStagesPer) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
@@ -485,7 +508,9 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
           const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
           if (contig_expert<CTAS>(tl, p) < 0) continue;
         }
-        if (!take(li)) continue;
+        int gb, ge;
+        if (!plan(li, gb, ge)) continue;
+        const int kb_hi = min(num_kb, 4 * ge);
         // one pipeline: alternate accumulators; two: accumulator = pipeline
         const uint32_t acc = PIPES == 2 ? pipe : (L::kNumAcc == 1 ? 0 : (own & 1));
         const uint32_t acc_use = (PIPES == 2 || L::kNumAcc == 1) ? own : (own >> 1);
@@ -496,7 +521,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
         uint32_t accumulate = 0;
-        for (int kb0 = kb_begin; kb0 < kb_end && ok; kb0 += 4, ++sf_group) {
+        for (int kb0 = 4 * gb; kb0 < kb_hi && ok; kb0 += 4, ++sf_group) {
           const uint32_t ring = sf_group % L::kSfRing;
           const uint32_t sf_col = sf_slot0 + (sf_group & 1) * L::kSfSlotCols;
           // TMEM scale slot (sf_group & 1) was last read by group sf_group - 2
@@ -519,7 +544,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
               tmem_cp_32x128b_warpx4<CTAS>(sf_col + 8, (static_cast<uint64_t>(sfx_hi) << 32) |
                                                            (lo + (L::kSftMainBytes >> 4)));
           }
-          const int nk = min(4, kb_end - kb0);
+          const int nk = min(4, kb_hi - kb0);
           uint32_t id = idesc0;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -572,10 +597,11 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       } else if (MODE == MODE_MASKED) {
         grp_a = grp_b = tl.g;
       }
-      if (!take(li)) continue;
+      int gb, ge;
+      if (!plan(li, gb, ge)) continue;
       const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
-      for (int kp = g_begin; kp < g_end; ++kp, ++group) {
+      for (int kp = gb; kp < ge; ++kp, ++group) {
         const uint32_t ring = group % L::kSfRing;
         ok = wait_phase<false>(&sf_empty[rbase + ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag);
         ok = __all_sync(0xffffffffu, ok);
@@ -645,6 +671,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     constexpr int kMaxMine = (kChunks + 1) / 2;
     const int nmine = half == 0 ? (kChunks + 1) / 2 : kChunks / 2;
     uint32_t local_tile = 0;
+    uint32_t uses0 = 0, uses1 = 0;  // tiles that used accumulator 0 / 1 so far (two pipelines)
     for (int t = unit0; t < ntiles; t += units) {
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
       int expert = 0, own_e = 0;
@@ -657,11 +684,20 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         expert = contig_expert<CTAS>(tl, p);
         if (expert < 0) continue;
       }
-      const uint32_t acc = SPLITK ? 0 : local_tile % L::kNumAcc;
-      const uint32_t acc_use = SPLITK ? local_tile : local_tile / L::kNumAcc;
+      // accumulator(s) of this tile and how often each was used before
+      uint32_t acc, acc_use;
+      bool split = false;
+      if constexpr (PIPES == 2) {
+        split = tile_split(local_tile);
+        acc = split ? 0u : static_cast<uint32_t>(tile_pipe(local_tile));
+        acc_use = acc == 0 ? uses0++ : uses1++;
+      } else {
+        acc = local_tile % L::kNumAcc;
+        acc_use = local_tile / L::kNumAcc;
+      }
       ++local_tile;
       bool ok = wait_phase<false>(&tmem_full[acc], acc_use & 1, abort_flag);
-      if (SPLITK && ok) ok = wait_phase<false>(&tmem_full[1], acc_use & 1, abort_flag);
+      if (split && ok) ok = wait_phase<false>(&tmem_full[1], uses1++ & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -767,24 +803,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         }
       };
 
-      if (SPLITK && any_valid) {
-        // sum of the two pipelines' accumulators, chunk by chunk
-        uint32_t r[2][32];
-#pragma unroll 1
-        for (int i = 0; i < nmine; ++i) {
-          const int c = half + 2 * i;
-          const int col0 = n0 + 32 * c;
-          if (col0 >= p.N) break;
-          tmem_ld_32x32b_x32(t_row + 32 * c, r[0]);
-          if (split_active) tmem_ld_32x32b_x32(t_row + L::kAccStride + 32 * c, r[1]);
-          tmem_wait_ld();
-          if (split_active) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) r[0][j] = __float_as_uint(__uint_as_float(r[0][j]) + __uint_as_float(r[1][j]));
-          }
-          store_chunk(r[0], col0);
-        }
-      } else if (any_valid) {
+      if (any_valid) {
         uint32_t r[2][32];
         if (nmine > 0 && n0 + 32 * half < p.N) tmem_ld_32x32b_x32(t_row + 32 * half, r[0]);
         tmem_wait_ld();
@@ -794,6 +813,19 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
           const int col0 = n0 + 32 * c;
           if (i >= nmine || col0 >= p.N) break;
           if (i + 1 < nmine && col0 + 64 < p.N) tmem_ld_32x32b_x32(t_row + 32 * (c + 2), r[(i + 1) & 1]);
+          if (split) {
+            // a split tile: add the second pipeline's accumulator, 16 columns at a time
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t h[16];
+              tmem_ld_32x32b_x16(t_row + L::kAccStride + 32 * c + 16 * hh, h);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                r[i & 1][16 * hh + j] =
+                    __float_as_uint(__uint_as_float(r[i & 1][16 * hh + j]) + __uint_as_float(h[j]));
+            }
+          }
           store_chunk(r[i & 1], col0);
           tmem_wait_ld();
         }
@@ -803,7 +835,10 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       if (lane == 0) {
         if constexpr (kPair) mbar_arrive_remote(empty0 + 8 * acc);
         else mbar_arrive(&tmem_empty[acc]);
-        if constexpr (SPLITK) mbar_arrive(&tmem_empty[1]);
+        if (split) {
+          if constexpr (kPair) mbar_arrive_remote(empty0 + 8);
+          else mbar_arrive(&tmem_empty[1]);
+        }
       }
     }
     if (lane == 0) bulk_wait_group<0>();

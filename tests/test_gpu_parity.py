@@ -276,3 +276,23 @@ def test_masked_is_graph_capturable_with_changing_counts():
         for gi, mg in enumerate(counts):
             check_close(got[gi, :mg], ref[gi, :mg], f"graph replay expert {gi}")
             assert (got[gi, mg:] == 0).all()
+
+
+@pytest.mark.parametrize("cfg", [(224, 2, 2), (128, 2, 2)])
+@pytest.mark.parametrize("K", [896, 1024, 2048])
+def test_odd_tile_count_splits_last_tile(cfg, K):
+    """With two pipelines a CTA whose tile count is odd splits its last tile
+    over both pipelines (each half of K, summed in the epilogue).  A small
+    grid (4 CTA pairs) gives every pair 3 tiles; K spans 2..4 scale groups,
+    with a ragged second half at K = 896."""
+    M, N = 512, 6 * cfg[0]
+    p = synth.dense_problem(M, N, K, seed=400 + K)
+    sa, sb = packed(p)
+    prev = dg.set_num_sms(8)
+    try:
+        dg.set_config(*cfg)
+        got = _run_dense(p, sa, sb)
+    finally:
+        dg.set_num_sms(prev)
+    check_close(got, oracle.fp8_gemm_nt(p.a, sa, p.b, sb, M, N, K), f"odd tiles cfg={cfg} K={K}")
+    assert dg.get_device_error() == 0
