@@ -176,8 +176,8 @@ static Config make_config() {
   c.bn = BN;
   c.stages = STAGES;
   c.ctas = CTAS;
-  c.smem = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>::kSmemBytes;
-  c.num_acc = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>::kNumAcc;
+  c.smem = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED>::kSmemBytes;
+  c.num_acc = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED>::kNumAcc;
   c.pipes = PIPES;
   c.layout = LAYOUT;
   c.splitk = SPLITK;
@@ -233,7 +233,7 @@ static const Config* config_table(int* count) {
         make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
         make_config<128, 6, MODE, 2>(), make_config<224, 6, MODE, 2>(), make_config<256, 6, MODE, 2>(),
         make_config<224, 6, MODE, 2, false, 2>(), make_config<128, 6, MODE, 2, false, 2>(),
-        make_config<64, 8, MODE, 1>(), make_config<64, 6, MODE, 1, false, 2, 0, true>(),
+        make_config<64, 8, MODE, 1>(), make_config<64, (MODE == MODE_DENSE ? 8 : 6), MODE, 1, false, 2, 0, true>(),
         make_config<128, 4, MODE, 1, false, 2, 0, true>(),
     };
     *count = static_cast<int>(sizeof(table) / sizeof(table[0]));

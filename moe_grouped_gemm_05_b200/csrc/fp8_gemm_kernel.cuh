@@ -111,7 +111,7 @@ struct GemmArgs {
   const float* c;     // optional FP32 addend [rows][N] (OUT_F32 only), nullptr for none
 };
 
-template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0>
+template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0, bool MASKED = true>
 struct Layout {
   static_assert(!(LAYOUT & 2) || (BN / CTAS) % 128 == 0, "an MN-major B tile is whole 128-column boxes per CTA");
   static_assert(CTAS == 1 || CTAS == 2, "CTAS is 1 or 2");
@@ -143,16 +143,19 @@ struct Layout {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSft = kOffB + STAGES * kBBytes;
+  // the masked layout's per-expert prefix and counts (other modes keep none)
+  static constexpr int kGroupsBytes = MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : 0;
   // scale ring depth (per pipeline): 4 groups when shared memory allows, else 2
   static constexpr int kSfRing =
-      (kOffSft + PIPES * 4 * kSftBytes + 1023) / 1024 * 1024 + 8 * kEpiBuf + 4096 +
-                  (2 * kMaxMaskedGroups + 1) * 4 + 1024 <= kMaxSmem ? 4 : 2;
+      (kOffSft + PIPES * 4 * kSftBytes + 1023) / 1024 * 1024 + 8 * kEpiBuf + 4096 + kGroupsBytes + 1024 <= kMaxSmem
+          ? 4
+          : 2;
   static constexpr int kOffEpi = ((kOffSft + PIPES * kSfRing * kSftBytes + 1023) / 1024) * 1024;
   static constexpr int kOffBar = kOffEpi + 8 * kEpiBuf;  // one staging buffer per epilogue warp
   static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 2 * PIPES * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag
   static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
-  static constexpr int kSmemBytes = kOffGroups + (2 * kMaxMaskedGroups + 1) * 4 + 1024;
+  static constexpr int kSmemBytes = kOffGroups + kGroupsBytes + 1024;
   static_assert(kSmemBytes <= kMaxSmem, "shared-memory budget exceeded");
   static_assert(kSfBaseCol + PIPES * 2 * kSfSlotCols <= kTmemCols, "TMEM budget exceeded");
 };
@@ -285,7 +288,7 @@ template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPE
 __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
-  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT>;
+  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED>;
   static_assert(LAYOUT == 0 || MODE == MODE_DENSE, "MN-major operands are built for the dense GEMM only");
   static_assert(!SPLITK || PIPES == 2, "split-K runs on two pipelines");
   constexpr bool kAmn = (LAYOUT & 1) != 0;
