@@ -84,3 +84,19 @@ def test_config_override(lib):
     assert lib.dg_set_config(224, 2, 0) == 0
     assert lib.dg_set_config(224, 2, 2) == 0
     assert lib.dg_set_config(0, 0, 0) == 0
+
+
+def test_heuristic_choices_without_gpu():
+    """The configuration heuristic is host logic: without a device it assumes
+    148 SMs.  Decode-sized dense problems take split-K tiles over two
+    pipelines, large ones 2-CTA tiles with two pipelines, masked problems
+    1-CTA tiles, and the pick is stable for the workloads the bench times."""
+    from moe_grouped_gemm_05_b200 import binding as dg
+
+    assert dg.describe_config("dense", 64, 7168, 2048).startswith("128x64x8(2pipe)(splitk)/112")
+    assert dg.describe_config("dense", 4096, 7168, 2048) == "256x224x6(2cta)(2pipe)/148"
+    assert dg.describe_config("dense", 8192, 8192, 8192) == "256x224x6(2cta)(2pipe)/148"
+    assert dg.describe_config("dense", 64, 7168, 512) == "128x64x8/112"  # one K group: no split
+    masked = dg.describe_config("masked", 256, 7168, 2048, 16)
+    assert "(2cta)" not in masked and masked.startswith("128x")
+    assert dg.describe_config("contiguous", 32768, 4096, 7168, 8) == "256x224x6(2cta)(2pipe)/148"
