@@ -484,285 +484,6 @@ def run_ours(args):
     e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1))
 
     flops = p.flops
-    return "tensor" if flops / algorithmic_bytes(p) > 560.0 else "hbm"
-
-
-def make_device_sets(p, dg, torch, dev):
-    """Device copies of one problem; enough copies that their total exceeds 2x L2."""
-    from moe_grouped_gemm_05_b200 import binding
-
-    a = torch.from_numpy(p.a).to(dev).view(torch.float8_e4m3fn)
-    b = torch.from_numpy(p.b).to(dev).view(torch.float8_e4m3fn)
-    sfa32 = torch.from_numpy(np.ascontiguousarray(p.sfa)).to(dev)
-    sfb32 = torch.from_numpy(np.ascontiguousarray(p.sfb)).to(dev)
-    if p.kind == "dense":
-        d_shape = (p.M, p.N)
-    elif p.kind == "contiguous":
-        d_shape = (p.M, p.N)
-    else:
-        d_shape = (p.G, p.M, p.N)
-    per_set = a.numel() + b.numel() + 2 * int(np.prod(d_shape))
-    nsets = max(1, -(-2 * L2_BYTES // per_set))
-    sets = []
-    for i in range(nsets):
-        s = {"a": a if i == 0 else a.clone(), "b": b if i == 0 else b.clone(),
-             "sfa32": sfa32 if i == 0 else sfa32.clone(),
-             "d": torch.empty(d_shape, dtype=torch.bfloat16, device=dev)}
-        s["sfb"] = binding.pack_sf_ue8m0(sfb32 if i == 0 else sfb32.clone())
-        s["sfa"] = binding.pack_sf_ue8m0(s["sfa32"])
-        if p.m_indices is not None:
-            s["m_indices"] = torch.from_numpy(p.m_indices).to(dev)
-        if p.masked_m is not None:
-            s["masked_m"] = torch.from_numpy(p.masked_m).to(dev)
-        sets.append(s)
-    return sets, per_set
-
-
-def gemm_call(p, dg, s, fp32_sfa=False):
-    """The GEMM of a step; with fp32_sfa it reads A's fp32 scales and packs them itself."""
-    sfa = s["sfa32"] if fp32_sfa else s["sfa"]
-    if p.kind == "dense":
-        return dg.fp8_gemm_nt(s["a"], sfa, s["b"], s["sfb"], s["d"])
-    if p.kind == "contiguous":
-        return dg.m_grouped_fp8_gemm_nt_contiguous(s["a"], sfa, s["b"], s["sfb"], s["m_indices"], s["d"])
-    return dg.m_grouped_fp8_gemm_nt_masked(s["a"], sfa, s["b"], s["sfb"], s["masked_m"], s["d"])
-
-
-def pack_call(dg, lib, s, torch):
-    """Packs the step's activation scales into s['sfa'] (the packing kernel, in place)."""
-    import ctypes
-
-    sf = s["sfa32"]
-    if sf.dim() == 2:
-        batch, mn, kb = 1, sf.shape[0], sf.shape[1]
-    else:
-        batch, mn, kb = sf.shape
-    code = lib.dg_pack_sf_ue8m0(ctypes.c_void_p(sf.data_ptr()), ctypes.c_void_p(s["sfa"].data_ptr()), batch, mn,
-                                kb, ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    if code != 0:
-        raise RuntimeError(lib.dg_get_last_error().decode())
-
-
-# ---------------------------------------------------------------- CPU oracle sample
-
-
-class OracleSample:
-    """The CPU oracle on a bounded row sample of a workload (all N, all K).
-
-    One run packs the sample rows' activation scales and computes their
-    output rows, i.e. the same two steps as one GPU step, on fewer rows."""
-
-    def __init__(self, p):
-        import oracle
-
-        self.oracle, self.p = oracle, p
-        if p.kind == "masked":
-            g = int(np.argmax(p.masked_m))
-            self.a, self.b, self.sfa32, sfb = p.a[g], p.b[g], p.sfa[g], p.sfb[g]
-            self.rows_total, self.desc = int(p.masked_m[g]), f"expert {g}"
-        elif p.kind == "contiguous":
-            self.a, self.b, self.sfa32, sfb = p.a, p.b[0], p.sfa, p.sfb[0]
-            self.rows_total, self.desc = int((p.m_indices == 0).sum()), "expert 0"
-        else:
-            self.a, self.b, self.sfa32, sfb = p.a, p.b, p.sfa, p.sfb
-            self.rows_total, self.desc = p.M, "the problem"
-        self.sfb = oracle.pack_sf_ue8m0(sfb[None])[0][0]  # weights: packed once
-        try:
-            from threadpoolctl import threadpool_info
-
-            self.cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-        except Exception:  # noqa: BLE001
-            self.cores = os.cpu_count() or 1
-
-    def run(self, rows: int) -> float:
-        p, o = self.p, self.oracle
-        t0 = time.perf_counter()
-        sfa = o.pack_sf_ue8m0(self.sfa32[None, :rows])[0][0]
-        o.fp8_gemm_nt(self.a[:rows], sfa, self.b, self.sfb, rows, p.N, p.K)
-        return time.perf_counter() - t0
-
-    def calibrate(self, seconds: float) -> int:
-        """Rows whose run takes about `seconds` (grown until a run is long enough to extrapolate)."""
-        rows = max(1, min(self.rows_total, 16))
-        while True:
-            t = self.run(rows)
-            if rows >= self.rows_total or t >= 0.25 * seconds:
-                break
-            rows = min(self.rows_total, rows * 4)
-        return int(max(1, min(self.rows_total, rows * seconds / max(t, 1e-6))))
-
-    def info(self, rows: int, t: float) -> dict:
-        p = self.p
-        return {"value": 2.0 * rows * p.N * p.K / t / 1e12, "unit": "TFLOPS", "cores": int(self.cores),
-                "kind": "oracle",
-                "sample": f"{p.name}: first {rows} valid rows of {self.desc} x all {p.N} columns x K={p.K}, "
-                          f"{t:.2f} s per run on host cores"}
-
-
-# ---------------------------------------------------------------- arms
-
-
-def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return 0
-    from moe_grouped_gemm_05_b200 import synth
-
-    p = synth.WORKLOADS[args.workload]()
-    total_steps = args.steps + args.warmup
-    per_step = max(0.05, min(2.0, 150.0 / max(total_steps, 1)))
-    smp = OracleSample(p)
-    rows = smp.calibrate(per_step)
-    times = []
-    for i in range(total_steps):
-        dt = smp.run(rows)
-        if i >= args.warmup:
-            times.append(dt)
-    step_s = statistics.mean(times) if times else smp.run(rows)
-    info = smp.info(rows, step_s)
-    value = info["value"]
-    line = {"metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload, "sample_rows": rows, "N": p.N, "K": p.K},
-            "impl": "reference", "cpu_baseline": info,
-            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
-    return 0
-
-
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
-
-    from moe_grouped_gemm_05_b200 import binding as dg
-    from moe_grouped_gemm_05_b200 import shard, synth
-
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus and world > 1:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    lib = dg.load()
-    # every rank runs its own copy of the problem: independent units, weak scaling
-    maker = synth.WORKLOADS[args.workload]
-    p = maker()
-    sets, per_set = make_device_sets(p, dg, torch, dev)
-    nsets = len(sets)
-    stream = torch.cuda.current_stream()
-
-    fused = args.fused_pack
-
-    def step(i):
-        s = sets[i % nsets]
-        if not fused:
-            pack_call(dg, lib, s, torch)
-        gemm_call(p, dg, s, fp32_sfa=fused)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    assert dg.get_device_error() == 0, "device error word set during warm-up"
-    kernel_desc = dg.describe_config(p.kind, p.M, p.N, p.K, p.G)
-
-    # The K timed steps are captured once as a CUDA graph and replayed, so the
-    # device runs them back to back without host launch gaps (--eager times
-    # host-issued launches instead).  A second graph holds the K GEMM launches
-    # alone and gives the kernel's own average duration.
-    cap = torch.cuda.Stream()
-    step_graph = gemm_graph = None
-    if not args.eager:
-        with torch.cuda.stream(cap):
-            cap.wait_stream(torch.cuda.current_stream())
-            step_graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(step_graph, stream=cap):
-                for i in range(args.steps):
-                    step(i)
-            gemm_graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gemm_graph, stream=cap):
-                for i in range(args.steps):
-                    gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
-        torch.cuda.synchronize()
-        step_graph.replay()  # upload + untimed pass
-        gemm_graph.replay()
-        torch.cuda.synchronize()
-    stream = torch.cuda.current_stream()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local).start()
-    barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    if step_graph is not None:
-        step_graph.replay()
-    else:
-        for i in range(args.steps):
-            step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    elapsed_ms = start.elapsed_time(end)
-    # kernel-only timing on the same stream, right after the timed region
-    g0 = torch.cuda.Event(enable_timing=True)
-    g1 = torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    if gemm_graph is not None:
-        gemm_graph.replay()
-    else:
-        for i in range(args.steps):
-            gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
-    g1.record(stream)
-    torch.cuda.synchronize()
-    sampler.stop()
-    gemm_avg_ms = g0.elapsed_time(g1) / args.steps
-    elapsed_ms = shard.max_over_ranks(elapsed_ms)
-    gemm_avg_ms = shard.max_over_ranks(gemm_avg_ms)
-    err = dg.get_device_error()
-
-    # end to end through the public API: pinned host inputs in, result out, every step
-    e2e_steps = args.e2e_steps or min(args.steps, 100)
-    s0 = sets[0]
-    a_host = torch.from_numpy(p.a).pin_memory()
-    sfa_host = torch.from_numpy(np.ascontiguousarray(p.sfa)).pin_memory()
-    d_host = torch.empty(s0["d"].shape, dtype=torch.bfloat16).pin_memory()
-    h2d = a_host.numel() + sfa_host.numel() * 4
-    d2h = d_host.numel() * 2
-    for _ in range(2):
-        s0["a"].view(torch.uint8).copy_(a_host, non_blocking=True)
-        s0["sfa32"].copy_(sfa_host, non_blocking=True)
-        if not fused:
-            pack_call(dg, lib, s0, torch)
-        gemm_call(p, dg, s0, fp32_sfa=fused)
-        d_host.copy_(s0["d"], non_blocking=True)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        s0["a"].view(torch.uint8).copy_(a_host, non_blocking=True)
-        s0["sfa32"].copy_(sfa_host, non_blocking=True)
-        if not fused:
-            pack_call(dg, lib, s0, torch)
-        gemm_call(p, dg, s0, fp32_sfa=fused)
-        d_host.copy_(s0["d"], non_blocking=True)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1))
-
-    flops = p.flops
     value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
     e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
