@@ -86,7 +86,7 @@ def test_config_override(lib):
     assert lib.dg_set_config(0, 0, 0) == 0
 
 
-def test_heuristic_choices_without_gpu():
+def test_heuristic_choices_without_gpu(lib):
     """The configuration heuristic is host logic: without a device it assumes
     148 SMs.  Decode-sized dense problems take split-K tiles over two
     pipelines, large ones 2-CTA tiles with two pipelines, masked problems
