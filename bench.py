@@ -68,18 +68,22 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+GEMM_KERNEL_SOURCES = ("fp8_gemm_kernel.cuh", "ptx.cuh")
+
+
 def kernel_source_hash() -> str:
+    """Hash of the GEMM kernel's device code (the host code is covered by the recorded configuration)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "moe_grouped_gemm_05_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in GEMM_KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, kernel_config: str):
     """Per-launch DRAM bytes of the GEMM kernel from a committed ncu summary,
-    only if it was taken on the current kernel sources."""
+    only if it was taken on the current kernel code in the same configuration."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
@@ -87,7 +91,7 @@ def recorded_traffic(workload: str):
     except (OSError, ValueError):
         return None
     ent = rec.get(workload)
-    if not ent or ent.get("kernel_hash") != kernel_source_hash():
+    if not ent or ent.get("kernel_hash") != kernel_source_hash() or ent.get("kernel_config") != kernel_config:
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -505,7 +509,7 @@ def run_ours(args):
         achieved = algorithmic_bytes(p) / (gemm_avg_ms * 1e-3) / 1e9
         unit = "GB/s"
         peak_note = f"copy bandwidth ({peak_src})"
-    traffic = recorded_traffic(args.workload)
+    traffic = recorded_traffic(args.workload, kernel_desc)
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,

@@ -235,6 +235,14 @@ int dg_get_device_error(void* stream, int* err);
 int dg_set_num_sms(int n);
 int dg_get_num_sms(void);
 
+/* Share of the GPU's tensor cores a call may occupy, in percent (1..100,
+ * 100 = all; the ssnai.com analysis lists set_tc_util beside set_num_sms
+ * and set_pdl as run-time tuning knobs, e.g. to leave SMs to a concurrent
+ * communication kernel).  Read here as a cap on the SMs a call plans and
+ * launches for: floor(SMs x percent / 100), at least one CTA pair, after
+ * dg_set_num_sms.  Returns the previous setting, or DG_ERR_SHAPE. */
+int dg_set_tc_util(int percent);
+
 /* Programmatic dependent launch for every kernel of this library (on by
  * default): a kernel's set-up (barrier init, tensor-memory allocation) may
  * overlap the end of the previous kernel on the stream; the kernel waits for

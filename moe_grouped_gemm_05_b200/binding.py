@@ -69,6 +69,7 @@ def load() -> ctypes.CDLL:
     lib.dg_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.dg_set_num_sms.argtypes = [i]
     lib.dg_set_pdl.argtypes = [i]
+    lib.dg_set_tc_util.argtypes = [i]
     lib.dg_get_num_sms.argtypes = []
     lib.dg_set_config.argtypes = [i, i, i]
     lib.dg_describe_config.argtypes = [i, i, i, i, i, ctypes.c_char_p, i]
@@ -345,6 +346,14 @@ def get_device_error() -> int:
 
 def set_num_sms(n: int) -> int:
     return load().dg_set_num_sms(n)
+
+
+def set_tc_util(percent: int) -> int:
+    """Caps the share of the GPU's SMs (tensor cores) a call may occupy; returns the previous percent."""
+    prev = load().dg_set_tc_util(percent)
+    if prev < 0:
+        _check(prev)
+    return prev
 
 
 def set_pdl(enable: bool) -> bool:

@@ -45,6 +45,17 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // ------------------------------------------------------------------ device info
 
 static int g_num_sms_override = 0;
+// Share of the GPU's tensor cores (SMs) a call may occupy, in percent.
+static std::atomic<int> g_tc_util{100};
+
+// SMs a call plans and launches for: the device's, capped by dg_set_num_sms
+// and by the dg_set_tc_util share (at least one CTA pair).
+static int usable_sms(int device_sms) {
+  int g = g_num_sms_override > 0 ? std::min(g_num_sms_override, device_sms) : device_sms;
+  const int u = g_tc_util.load(std::memory_order_relaxed);
+  if (u < 100) g = std::max(2, g * u / 100);
+  return g;
+}
 // Programmatic dependent launch of every kernel (on by default): a kernel may
 // start its set-up while the previous grid of the stream finishes, and waits
 // (griddepcontrol.wait) before its first global-memory access.
@@ -494,7 +505,7 @@ static int check_common(const void* a, const void* sfa, const void* b, const int
 // Persistent grid: one CTA per SM (co-resident pairs for 2-CTA tiles), never
 // more units than tiles.
 static int grid_size(int sms, long long tiles, const Config* cfg) {
-  int g = g_num_sms_override > 0 ? std::min(g_num_sms_override, sms) : sms;
+  const int g = usable_sms(sms);
   long long units = g / cfg->ctas;
   if (cfg->ctas == 2) units = std::min<long long>(units, max_active_pairs(cfg, sms));
   if (tiles < units) units = std::max<long long>(tiles, 1);
@@ -547,7 +558,7 @@ static int gemm_dense(const void* a, const void* sfa, const void* b, const int32
   }
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const Config* cfg = choose_config<HMODE>(M, N, K, di.sms);
+  const Config* cfg = choose_config<HMODE>(M, N, K, usable_sms(di.sms));
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
   if ((r = build_maps_cached(maps, cfg, a, b, d, M, 1, N, K, 1, M, 1))) return r;
@@ -584,6 +595,11 @@ int dg_set_num_sms(int n) {
 
 int dg_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0); }
 
+int dg_set_tc_util(int percent) {
+  if (percent < 1 || percent > 100) return fail(DG_ERR_SHAPE, "percent=%d must be in [1, 100]", percent);
+  return g_tc_util.exchange(percent);
+}
+
 int dg_get_num_sms(void) {
   DeviceInfo di;
   if (device_info(&di) != DG_OK) return g_num_sms_override;
@@ -612,7 +628,8 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
   DeviceInfo di;
   int sms = 148;
   if (device_info(&di) == DG_OK) sms = di.sms;
-  if (g_num_sms_override > 0) sms = std::min(sms, g_num_sms_override);
+  const int device_sms = sms;
+  sms = usable_sms(sms);
   if (N <= 0 || K <= 0) return fail(DG_ERR_SHAPE, "N and K must be positive");
   const Config* c = nullptr;
   long long tiles = 0;
@@ -626,7 +643,7 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
   }
   if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
   snprintf(buf, buflen, "%dx%dx%d%s%s%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
-           c->pipes == 2 ? "(2pipe)" : "", c->splitk ? "(splitk)" : "", grid_size(sms, tiles, c));
+           c->pipes == 2 ? "(2pipe)" : "", c->splitk ? "(splitk)" : "", grid_size(device_sms, tiles, c));
   return DG_OK;
 }
 
@@ -781,7 +798,7 @@ int dg_fp8_gemm_nt_ex(const void* a, const int32_t* sfa, const void* b, const in
   if (M == 0) return DG_OK;
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const Config* cfg = d_is_fp32 ? choose_config<MODE_DENSE_F32>(M, N, K, di.sms) : choose_config<MODE_DENSE>(M, N, K, di.sms);
+  const Config* cfg = d_is_fp32 ? choose_config<MODE_DENSE_F32>(M, N, K, usable_sms(di.sms)) : choose_config<MODE_DENSE>(M, N, K, usable_sms(di.sms));
   if (!cfg && d_is_fp32) cfg = find_config<MODE_DENSE_F32>(224, 1);  // forced 2-CTA configs have no FP32 form
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
@@ -816,7 +833,7 @@ static int contiguous_impl(const void* a, const void* sfa, const void* b, const 
   if (M_total == 0) return DG_OK;
   DeviceInfo di;
   if ((r = device_info(&di))) return r;
-  const Config* cfg = choose_config<MODE_CONTIG>(M_total, N, K, di.sms, num_groups);
+  const Config* cfg = choose_config<MODE_CONTIG>(M_total, N, K, usable_sms(di.sms), num_groups);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
   if ((r = build_maps_cached(maps, cfg, a, b, d, M_total, 1, N, K, num_groups, M_total, 1))) return r;
@@ -862,7 +879,7 @@ static int masked_impl(const void* a, const void* sfa, const void* b, const int3
   if ((r = device_info(&di))) return r;
   // the device decides the real tile count; the heuristic assumes half-full experts
   const long long rows_est = std::max<long long>(1, static_cast<long long>(num_groups) * M_max / 2);
-  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, di.sms);
+  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, usable_sms(di.sms));
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
   if ((r = build_maps_cached(maps, cfg, a, b, d, M_max, num_groups, N, K, num_groups, M_max, num_groups)))

@@ -100,3 +100,16 @@ def test_heuristic_choices_without_gpu(lib):
     masked = dg.describe_config("masked", 256, 7168, 2048, 16)
     assert "(2cta)" not in masked and masked.startswith("128x")
     assert dg.describe_config("contiguous", 32768, 4096, 7168, 8) == "256x224x6(2cta)(2pipe)/148"
+
+
+def test_tc_util_caps_the_planned_grid(lib):
+    from moe_grouped_gemm_05_b200 import binding as dg
+
+    assert lib.dg_set_tc_util(0) == -2 and lib.dg_set_tc_util(101) == -2
+    assert dg.set_tc_util(50) == 100
+    try:
+        desc = dg.describe_config("dense", 4096, 7168, 2048)
+        assert int(desc.split("/")[-1]) <= 74, desc
+    finally:
+        assert dg.set_tc_util(100) == 50
+    assert dg.describe_config("dense", 4096, 7168, 2048).endswith("/148")
