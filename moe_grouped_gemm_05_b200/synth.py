@@ -190,6 +190,9 @@ class Problem:
 
     @property
     def flops(self) -> float:
+        """Algorithmic work, 2*M*N*K with M the valid rows only (discosf.com
+        DeepGEMM tutorial, section 4.3: one multiply and one add per term;
+        padding and masked-out rows do no useful work and are not counted)."""
         return 2.0 * self.valid_rows * self.N * self.K
 
 

@@ -40,6 +40,8 @@ BLOCK = 128
 def e4m3_table() -> np.ndarray:
     """Value of each of the 256 E4M3 ("E4M3FN") codes as float64.
 
+    discosf.com DeepGEMM tutorial, section 2.3 (E4M3: 4 exponent and 3
+    mantissa bits) and the float8_e4m3fn dtype of its section 4.2 example.
     Sign bit 7, exponent bits 6..3 (bias 7), mantissa bits 2..0.  Exponent 0
     encodes subnormals m/8 * 2^-6; S.1111.111 is NaN; there is no infinity, so
     the largest finite magnitude is 1.75 * 2^8 = 448.
