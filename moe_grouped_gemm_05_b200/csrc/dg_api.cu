@@ -44,14 +44,15 @@ static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 // ------------------------------------------------------------------ device info
 
-static int g_num_sms_override = 0;
+static std::atomic<int> g_num_sms_override{0};
 // Share of the GPU's tensor cores (SMs) a call may occupy, in percent.
 static std::atomic<int> g_tc_util{100};
 
 // SMs a call plans and launches for: the device's, capped by dg_set_num_sms
 // and by the dg_set_tc_util share (at least one CTA pair).
 static int usable_sms(int device_sms) {
-  int g = g_num_sms_override > 0 ? std::min(g_num_sms_override, device_sms) : device_sms;
+  const int o = g_num_sms_override.load(std::memory_order_relaxed);
+  int g = o > 0 ? std::min(o, device_sms) : device_sms;
   const int u = g_tc_util.load(std::memory_order_relaxed);
   if (u < 100) g = std::max(2, g * u / 100);
   return g;
@@ -359,20 +360,24 @@ static int max_active_pairs(const Config* cfg, int sms) {
 template <int MODE>
 static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const GemmArgs& args,
                   cudaStream_t stream) {
+  // The shared-memory opt-in is a per-device function attribute: set it once
+  // per (device, configuration).
+  constexpr int kMaxDevices = 64, kMaxConfigs = 32;
   static std::mutex mu;
-  static bool attr_done[32] = {};
-  int idx = 0;
-  {
-    int n = 0;
-    const Config* t = config_table<MODE>(&n);
-    idx = static_cast<int>(cfg - t);
-  }
+  static bool attr_done[kMaxDevices][kMaxConfigs] = {};
+  int n = 0;
+  const Config* t = config_table<MODE>(&n);
+  const int idx = static_cast<int>(cfg - t);
+  int dev = 0;
+  DG_CUDA_TRY(cudaGetDevice(&dev));
+  if (idx < 0 || idx >= n || idx >= kMaxConfigs || dev < 0 || dev >= kMaxDevices)
+    return fail(DG_ERR_UNSUPPORTED, "configuration %d / device %d outside the launch table", idx, dev);
   {
     std::lock_guard<std::mutex> lock(mu);
-    if (!attr_done[idx]) {
+    if (!attr_done[dev][idx]) {
       DG_CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(cfg->fn),
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, cfg->smem));
-      attr_done[idx] = true;
+      attr_done[dev][idx] = true;
     }
   }
   LaunchAttrs la(cfg->ctas);
@@ -588,9 +593,7 @@ int64_t dg_packed_sf_words(int mn, int kb) {
 const char* dg_get_last_error(void) { return t_last_error; }
 
 int dg_set_num_sms(int n) {
-  const int prev = g_num_sms_override;
-  g_num_sms_override = n > 0 ? n : 0;
-  return prev;
+  return g_num_sms_override.exchange(n > 0 ? n : 0);
 }
 
 int dg_set_pdl(int enable) { return g_pdl.exchange(enable ? 1 : 0); }
@@ -602,8 +605,9 @@ int dg_set_tc_util(int percent) {
 
 int dg_get_num_sms(void) {
   DeviceInfo di;
-  if (device_info(&di) != DG_OK) return g_num_sms_override;
-  return g_num_sms_override > 0 ? std::min(g_num_sms_override, di.sms) : di.sms;
+  const int o = g_num_sms_override.load(std::memory_order_relaxed);
+  if (device_info(&di) != DG_OK) return o;
+  return o > 0 ? std::min(o, di.sms) : di.sms;
 }
 
 int dg_set_config(int block_n, int ctas, int pipes) {
