@@ -138,3 +138,81 @@ def test_gemm_worked_example():
         m, n = int(m), int(n)
         assert Fraction(exact[m, n]) == Fraction(val), (m, n, exact[m, n])
         assert bits[m, n] == int(bf, 16), (m, n, hex(bits[m, n]))
+
+
+SENTINEL = 0xDEAD
+
+
+def _grouped_inputs(sec):
+    G = 1 + max(int(f[0]) for f in sec["experts"])
+    b = np.zeros((G, 2, 128), np.uint8)
+    for e, n, code in sec["experts"]:
+        b[int(e), int(n)] = int(code, 16)
+    sfb = np.concatenate([_words([[int(x)]], 1) for _, x in sorted(sec["sfb"], key=lambda f: int(f[0]))])
+    return G, b, sfb
+
+
+def _check_d(d, rows_expected, key_len):
+    written = set()
+    for f in rows_expected:
+        idx = tuple(int(x) for x in f[:key_len])
+        v0, v1, b0, b1 = f[key_len:]
+        assert d[idx].tolist() == [int(b0, 16), int(b1, 16)], (idx, [hex(x) for x in d[idx]])
+        assert Fraction(float(oracle.bf16_bits_to_f64(d[idx])[0])) == Fraction(v0)
+        assert Fraction(float(oracle.bf16_bits_to_f64(d[idx])[1])) == Fraction(v1)
+        written.add(idx)
+    return written
+
+
+def test_contiguous_worked_example():
+    sec = _sections("grouped_worked_example.txt")
+    G, b, sfb = _grouped_inputs(sec)
+    rows = sec["contiguous"]
+    M = len(rows)
+    a = np.stack([np.full(128, int(code, 16), np.uint8) for _, code, _, _ in rows])
+    sfa = _words([[int(x)] for _, _, x, _ in rows], M)
+    m_idx = np.array([int(f[3]) for f in rows], np.int32)
+
+    d = np.full((M, 2), SENTINEL, np.uint16)
+    assert oracle.m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_idx, d, G, 2, 128) == 0
+    written = _check_d(d, sec["contiguous_d"], 1)
+    for m in range(M):
+        if (m,) not in written:
+            assert (d[m] == SENTINEL).all(), m
+
+    kind, row, index, reported = next(f for f in sec["errors"] if f[0] == "contiguous_index")
+    bad_idx = m_idx.copy()
+    bad_idx[int(row)] = int(index)
+    d2 = np.full((M, 2), SENTINEL, np.uint16)
+    assert oracle.m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, bad_idx, d2, G, 2, 128) == int(reported)
+    assert (d2[int(row)] == SENTINEL).all()
+    others = [m for m in range(M) if m != int(row)]
+    assert np.array_equal(d2[others], d[others])
+
+
+def test_masked_worked_example():
+    sec = _sections("grouped_worked_example.txt")
+    G, b, sfb = _grouped_inputs(sec)
+    M_max = 1 + max(int(f[1]) for f in sec["masked"])
+    a = np.zeros((G, M_max, 128), np.uint8)
+    ea = [[[0] for _ in range(M_max)] for _ in range(G)]
+    for g, r, code, x in sec["masked"]:
+        a[int(g), int(r)] = int(code, 16)
+        ea[int(g)][int(r)] = [int(x)]
+    sfa = np.concatenate([_words(ea[g], M_max) for g in range(G)])
+    mm = np.array([int(x) for x in sec["masked_m"][0]], np.int32)
+
+    d = np.full((G, M_max, 2), SENTINEL, np.uint16)
+    assert oracle.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, mm, d, G, M_max, 2, 128) == 0
+    written = _check_d(d, sec["masked_d"], 2)
+    for g in range(G):
+        for r in range(M_max):
+            if (g, r) not in written:
+                assert (d[g, r] == SENTINEL).all(), (g, r)
+
+    kind, g, count, reported = next(f for f in sec["errors"] if f[0] == "masked_count")
+    mm2 = mm.copy()
+    mm2[int(g)] = int(count)
+    d2 = np.full((G, M_max, 2), SENTINEL, np.uint16)
+    assert oracle.m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, mm2, d2, G, M_max, 2, 128) == int(reported)
+    assert np.array_equal(d2, d)
