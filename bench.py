@@ -165,16 +165,20 @@ class ClockSampler:
 
 
 def algorithmic_bytes(p) -> float:
-    """Bytes the GEMM must move at least once: A rows read, B read, D written, scales."""
+    """Bytes the GEMM must move at least once: the valid A rows read, B read for
+    every expert that has rows, the valid D rows written (BF16), and one UE8M0
+    byte per scale of those A rows and B blocks.  Padding and masked-out rows
+    cost nothing here, as they do nothing useful."""
     kb = p.K // 128
+    nb = (p.N + 127) // 128
+    rows = p.valid_rows
     if p.kind == "dense":
-        return p.M * p.K + p.N * p.K + 2.0 * p.M * p.N + 4.0 * (p.M + (p.N + 127) // 128) * kb / 4
-    if p.kind == "contiguous":
-        v = p.valid_rows
-        return v * p.K + p.G * p.N * p.K + 2.0 * v * p.N
-    v = p.valid_rows
-    active = int((p.masked_m > 0).sum())
-    return v * p.K + active * p.N * p.K + 2.0 * v * p.N
+        experts = 1
+    elif p.kind == "contiguous":
+        experts = len(np.unique(p.m_indices[p.m_indices >= 0]))
+    else:
+        experts = int((p.masked_m > 0).sum())
+    return rows * (p.K + kb) + experts * (p.N * p.K + nb * kb) + 2.0 * rows * p.N
 
 
 def bound_of(p) -> str:
