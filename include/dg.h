@@ -211,7 +211,10 @@ int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int 
  * num_experts <= 1024; M_cap >= dg_moe_permute_capacity(...) and a multiple of 128.
  * dg_moe_unpermute_combine:
  *   out[t] = bf16_rne( sum_s weights[t][s] * d_perm[row_of[t][s]] ) in FP32 over routed
- *   slots (weights NULL = 1); d_perm BF16 [>= rows][N], out BF16 [T][N], N % 16 == 0.
+ *   slots (weights NULL = 1); d_perm BF16 [rows][N], out BF16 [T][N], N % 16 == 0.
+ *   Every row_of entry must be -1 or a row of d_perm.  The call has no row count of
+ *   d_perm to check them against (row_of is device data), so this is the caller's
+ *   contract; row_of from dg_moe_permute with d_perm of M_cap rows meets it.
  */
 int dg_moe_permute_capacity(int T, int topk, int num_experts);
 int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, const void* q, const int32_t* sfa, int K,

@@ -122,6 +122,30 @@ def packed_sf_words(mn: int, kb: int) -> tuple[int, int]:
     return (kb + 3) // 4, (mn + 3) // 4 * 4
 
 
+def _packed_numel(t, batch: int, mn: int, kb: int, name: str):
+    """Packed scale words may come as [kp, mn4] or [batch, kp, mn4]: what the
+    kernels read is batch * kp * mn4 words, so the element count must match."""
+    kp, mn4 = packed_sf_words(mn, kb)
+    if t.numel() != batch * kp * mn4:
+        raise ValueError(f"{name} holds {t.numel()} words; expected {batch} x {kp} x {mn4} "
+                         f"(batch x ceil(Kb/4) x align4(MN))")
+
+
+def _same_device(ref, *tensors):
+    """All operands of a call live on one device (None entries are skipped)."""
+    dev = ref.get_device()
+    for t in tensors:
+        if t is not None and t.get_device() != dev:
+            raise ValueError(f"operands on different devices: {ref.device} and {t.device}")
+
+
+def _out(t, dtypes, shape, name: str, device):
+    """Checks a caller-provided output tensor."""
+    if t.dtype not in dtypes or tuple(t.shape) != tuple(shape) or not t.is_contiguous() or t.device != device:
+        raise ValueError(f"{name} must be a contiguous {'/'.join(str(d) for d in dtypes)} tensor of shape "
+                         f"{tuple(shape)} on {device}")
+
+
 def pack_sf_ue8m0(sf: torch.Tensor, out=None) -> torch.Tensor:
     """fp32 power-of-two scales [batch?, mn, kb] -> int32 [batch?, ceil(kb/4), align4(mn)] (into `out` if given)."""
     if sf.dtype != torch.float32 or not sf.is_cuda or not sf.is_contiguous():
@@ -134,8 +158,9 @@ def pack_sf_ue8m0(sf: torch.Tensor, out=None) -> torch.Tensor:
     kp, mn4 = packed_sf_words(mn, kb)
     if out is None:
         out = torch.empty((batch, kp, mn4), dtype=torch.int32, device=sf.device)
-    elif out.dtype != torch.int32 or not out.is_contiguous() or out.numel() != batch * kp * mn4:
-        raise ValueError("out must be a contiguous int32 tensor of the packed shape")
+    elif (out.dtype != torch.int32 or not out.is_contiguous() or out.numel() != batch * kp * mn4
+          or out.device != sf.device):
+        raise ValueError("out must be a contiguous int32 tensor of the packed shape on sf's device")
     _check(load().dg_pack_sf_ue8m0(_ptr(s3), _ptr(out), batch, mn, kb, _stream()))
     if out.dim() == 3 and squeeze:
         return out[0]
@@ -161,8 +186,8 @@ def quantize_fp8_1x128(x: torch.Tensor, q=None, sf=None):
         q = torch.empty(x.shape, dtype=torch.float8_e4m3fn, device=x.device)
     if sf is None:
         sf = torch.empty((*lead, kp, mn4), dtype=torch.int32, device=x.device)
-    if tuple(q.shape) != tuple(x.shape) or tuple(sf.shape) != (*lead, kp, mn4):
-        raise ValueError("q / sf shapes do not match x")
+    _out(q, (torch.float8_e4m3fn, torch.uint8), x.shape, "q", x.device)
+    _out(sf, (torch.int32,), (*lead, kp, mn4), "sf", x.device)
     _check(load().dg_quantize_fp8_1x128(_ptr(x), 0 if x.dtype == torch.bfloat16 else 1, _ptr(q), _ptr(sf), batch,
                                         M, K, _stream()))
     return q, sf
@@ -193,6 +218,7 @@ def fp8_gemm_nt(a, sfa, b, sfb, d=None) -> torch.Tensor:
     if (not fp32_sfa and tuple(sfa.shape) != packed_sf_words(M, K // 128)) or \
             tuple(sfb.shape) != packed_sf_words(-(-N // 128), K // 128):
         raise ValueError("packed scale shapes do not match [ceil(Kb/4), align4(MN)]")
+    _same_device(a, sfa, b, sfb, d)
     if d is None:
         d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
@@ -219,6 +245,7 @@ def fp8_gemm(layout: str, a, sfa, b, sfb, d=None) -> torch.Tensor:
         raise ValueError("a and b disagree on K")
     if tuple(sfa.shape) != packed_sf_words(M, K // 128) or tuple(sfb.shape) != packed_sf_words(-(-N // 128), K // 128):
         raise ValueError("packed scale shapes do not match [ceil(Kb/4), align4(MN)]")
+    _same_device(a, sfa, b, sfb, d)
     if d is None:
         d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
@@ -242,8 +269,13 @@ def fp8_gemm_nt_ex(a, sfa, b, sfb, c=None, d=None, recipe_b: int = 128, out_dtyp
         raise ValueError("packed scale shapes do not match the recipe")
     if c is not None and (c.dtype != torch.float32 or tuple(c.shape) != (M, N) or not c.is_contiguous()):
         raise ValueError("c must be a contiguous float32 [M, N] tensor")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    _same_device(a, sfa, b, sfb, c, d)
     if d is None:
         d = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    else:
+        _out(d, (torch.bfloat16, torch.float32), (M, N), "d", a.device)
     _check(load().dg_fp8_gemm_nt_ex(_ptr(a), _ptr(sfa), _ptr(b), _ptr(sfb), _ptr(c) if c is not None else None,
                                     _ptr(d), M, N, K, recipe_b, 1 if d.dtype == torch.float32 else 0, _stream()))
     return d
@@ -259,6 +291,10 @@ def m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, m_indices, d=None) -> torch
     if Kb_ != K or m_indices.shape != (M,):
         raise ValueError("shape mismatch")
     fp32_sfa = _sfa_kind(sfa, (M,), K)
+    if not fp32_sfa:
+        _packed_numel(sfa, 1, M, K // 128, "sfa")
+    _packed_numel(sfb, G, -(-N // 128), K // 128, "sfb")
+    _same_device(a, sfa, b, sfb, m_indices, d)
     if d is None:
         d = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (M, N) or not d.is_contiguous():
@@ -278,6 +314,10 @@ def m_grouped_fp8_gemm_nt_masked(a, sfa, b, sfb, masked_m, d=None) -> torch.Tens
     if Gb != G or Kb_ != K or masked_m.shape != (G,):
         raise ValueError("shape mismatch")
     fp32_sfa = _sfa_kind(sfa, (G, M_max), K)
+    if not fp32_sfa:
+        _packed_numel(sfa, G, M_max, K // 128, "sfa")
+    _packed_numel(sfb, G, -(-N // 128), K // 128, "sfb")
+    _same_device(a, sfa, b, sfb, masked_m, d)
     if d is None:
         d = torch.empty((G, M_max, N), dtype=torch.bfloat16, device=a.device)
     elif d.dtype != torch.bfloat16 or tuple(d.shape) != (G, M_max, N) or not d.is_contiguous():
@@ -296,7 +336,11 @@ def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: 
     """
     _i32(topk_ids, "topk_ids"), _fp8(q, "q"), _i32(sfa, "sfa")
     T, topk = topk_ids.shape
+    if q.dim() != 2 or q.shape[0] != T:
+        raise ValueError(f"q must be [T, K] with T = {T} rows, one per token of topk_ids")
     K = q.shape[1]
+    _packed_numel(sfa, 1, T, K // 128, "sfa")
+    _same_device(q, topk_ids, sfa)
     cap = load().dg_moe_permute_capacity(T, topk, num_experts)
     if cap < 0:
         _check(cap)
@@ -311,10 +355,13 @@ def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: 
             "row_of": torch.empty((T, topk), dtype=torch.int32, device=dev),
         }
     else:
-        want = {"a": (cap, K), "sfa": (kp, cap), "m_indices": (cap,), "src_of": (cap,), "row_of": (T, topk)}
-        for key, shape in want.items():
-            if key not in out or tuple(out[key].shape) != shape or not out[key].is_contiguous():
-                raise ValueError(f"out[{key!r}] must be a contiguous tensor of shape {shape}")
+        want = {"a": ((torch.float8_e4m3fn, torch.uint8), (cap, K)), "sfa": ((torch.int32,), (kp, cap)),
+                "m_indices": ((torch.int32,), (cap,)), "src_of": ((torch.int32,), (cap,)),
+                "row_of": ((torch.int32,), (T, topk))}
+        for key, (dtypes, shape) in want.items():
+            if key not in out:
+                raise ValueError(f"out[{key!r}] is missing")
+            _out(out[key], dtypes, shape, f"out[{key!r}]", dev)
     _check(load().dg_moe_permute(_ptr(topk_ids), T, topk, num_experts, _ptr(q), _ptr(sfa), K, _ptr(out["a"]),
                                  _ptr(out["sfa"]), _ptr(out["m_indices"]), _ptr(out["row_of"]), _ptr(out["src_of"]),
                                  cap, _stream()))
@@ -323,15 +370,18 @@ def moe_permute(topk_ids: torch.Tensor, num_experts: int, q: torch.Tensor, sfa: 
 
 def moe_unpermute_combine(d_perm: torch.Tensor, row_of: torch.Tensor, weights=None, out=None) -> torch.Tensor:
     """out[t] = sum_s weights[t, s] * d_perm[row_of[t, s]] (bf16, FP32 sums)."""
-    if d_perm.dtype != torch.bfloat16 or not d_perm.is_contiguous():
-        raise TypeError("d_perm must be contiguous bf16")
+    if d_perm.dtype != torch.bfloat16 or not d_perm.is_contiguous() or not d_perm.is_cuda or d_perm.dim() != 2:
+        raise TypeError("d_perm must be a contiguous bf16 [rows, N] CUDA tensor")
     _i32(row_of, "row_of")
     T, topk = row_of.shape
     N = d_perm.shape[1]
-    if weights is not None and (weights.dtype != torch.float32 or tuple(weights.shape) != (T, topk)):
-        raise ValueError("weights must be float32 [T, topk]")
+    if weights is not None:
+        _out(weights, (torch.float32,), (T, topk), "weights", d_perm.device)
+    _same_device(d_perm, row_of)
     if out is None:
         out = torch.empty((T, N), dtype=torch.bfloat16, device=d_perm.device)
+    else:
+        _out(out, (torch.bfloat16,), (T, N), "out", d_perm.device)
     _check(load().dg_moe_unpermute_combine(_ptr(d_perm), _ptr(row_of), _ptr(weights) if weights is not None else None,
                                            T, topk, N, _ptr(out), _stream()))
     return out

@@ -113,3 +113,38 @@ def test_tc_util_caps_the_planned_grid(lib):
     finally:
         assert dg.set_tc_util(100) == 50
     assert dg.describe_config("dense", 4096, 7168, 2048).endswith("/148")
+
+
+def test_binding_argument_helpers_without_gpu():
+    """The binding's checks that keep a wrongly sized tensor from reaching a
+    kernel: packed scale element counts, one device for all operands, and
+    caller-provided outputs."""
+    import torch
+
+    from moe_grouped_gemm_05_b200 import binding as dg
+
+    # [kp, mn4] or [batch, kp, mn4]: ceil(5/4) = 2, align4(5) = 8
+    dg._packed_numel(torch.empty(2, 8, dtype=torch.int32), 1, 5, 5, "sfa")
+    dg._packed_numel(torch.empty(3, 2, 8, dtype=torch.int32), 3, 5, 5, "sfb")
+    with pytest.raises(ValueError, match="expected 3 x 2 x 8"):
+        dg._packed_numel(torch.empty(2, 8, dtype=torch.int32), 3, 5, 5, "sfb")
+    with pytest.raises(ValueError):
+        dg._packed_numel(torch.empty(1, 8, dtype=torch.int32), 1, 5, 5, "sfa")   # one K word short
+
+    x = torch.empty(4)
+    dg._same_device(x, torch.empty(2), None)
+    from types import SimpleNamespace
+    other = SimpleNamespace(get_device=lambda: 1, device="cuda:1")   # stands in for a tensor on GPU 1
+    with pytest.raises(ValueError, match="cuda:1"):
+        dg._same_device(x, torch.empty(2), other)
+
+    out = torch.empty(3, 4, dtype=torch.bfloat16)
+    dg._out(out, (torch.bfloat16,), (3, 4), "out", out.device)
+    with pytest.raises(ValueError):
+        dg._out(out, (torch.float32,), (3, 4), "out", out.device)         # dtype
+    with pytest.raises(ValueError):
+        dg._out(out, (torch.bfloat16,), (4, 3), "out", out.device)        # shape
+    with pytest.raises(ValueError):
+        dg._out(out.t(), (torch.bfloat16,), (4, 3), "out", out.device)    # not contiguous
+    with pytest.raises(ValueError):
+        dg._out(out, (torch.bfloat16,), (3, 4), "out", torch.device("meta"))
