@@ -52,6 +52,34 @@ def partition_experts(rows_per_expert, world: int) -> list[list[int]]:
     return [sorted(o) for o in owned]
 
 
+def local_contiguous_layout(m_indices, owned, align: int = 128):
+    """This rank's contiguous layout when it owns the experts in ``owned``.
+
+    The owned experts' rows are taken from the global contiguous layout in
+    expert order (the order of ``owned``), keeping their order within each
+    expert, and each expert's segment is padded with -1 to a multiple of
+    ``align`` rows.  Returns ``(src_rows, local_m_indices)``, both int32 of
+    the local row count: ``src_rows[i]`` is the global row that local row ``i``
+    holds (-1 for padding), and ``local_m_indices[i]`` its expert's position
+    in ``owned`` (-1 for padding).  Scattering the local output rows back to
+    ``src_rows`` reproduces the global output of those experts.
+    """
+    m_indices = np.asarray(m_indices)
+    src, loc = [], []
+    for j, g in enumerate(owned):
+        rows = np.nonzero(m_indices == g)[0]
+        padded = -(-len(rows) // align) * align
+        seg_src = np.full(padded, -1, np.int32)
+        seg_src[:len(rows)] = rows
+        seg_loc = np.full(padded, -1, np.int32)
+        seg_loc[:len(rows)] = j
+        src.append(seg_src)
+        loc.append(seg_loc)
+    if not src:
+        return np.zeros(0, np.int32), np.zeros(0, np.int32)
+    return np.concatenate(src), np.concatenate(loc)
+
+
 def max_over_ranks(value: float, group=None) -> float:
     """Maximum of `value` over all ranks of the default process group (identity when not distributed)."""
     import torch

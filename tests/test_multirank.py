@@ -84,6 +84,53 @@ def _rank_dense(rank, world):
     return gathered
 
 
+def _rank_contiguous(rank, world):
+    counts = [300, 0, 40, 128, 77]
+    p = synth.contiguous_problem(5, 256, 256, rows=0, seed=53, counts=counts)
+    owned = shard.partition_experts(counts, world)[rank]
+    src, loc = shard.local_contiguous_layout(p.m_indices, owned)
+    take = np.maximum(src, 0)
+    a = p.a[take]                                   # padding rows: any bytes, never read into D
+    sa, _ = oracle.pack_sf_ue8m0(p.sfa[take][None])
+    sb, _ = oracle.pack_sf_ue8m0(p.sfb[owned]) if owned else (np.zeros((0, 1, 4), np.int32), 0)
+    d_local = np.zeros((len(src), p.N), np.uint16)
+    if owned:
+        assert oracle.m_grouped_fp8_gemm_nt_contiguous(a, sa[0], p.b[owned], sb, loc, d_local, len(owned),
+                                                       p.N, p.K) == 0
+    d = np.zeros((p.M, p.N), np.uint16)
+    d[src[src >= 0]] = d_local[src >= 0]
+    gathered = [None] * world
+    dist.all_gather_object(gathered, (owned, d, len(src) % 128))
+    return gathered
+
+
+@pytest.mark.timeout(300)
+def test_expert_parallel_contiguous_equals_unsharded():
+    gathered = _run(_rank_contiguous)[0]
+    p = synth.contiguous_problem(5, 256, 256, rows=0, seed=53, counts=[300, 0, 40, 128, 77])
+    sa, _ = oracle.pack_sf_ue8m0(p.sfa[None])
+    sb, _ = oracle.pack_sf_ue8m0(p.sfb)
+    ref = np.zeros((p.M, p.N), np.uint16)
+    assert oracle.m_grouped_fp8_gemm_nt_contiguous(p.a, sa[0], p.b, sb, p.m_indices, ref, p.G, p.N, p.K) == 0
+    assert sorted(g for owned, _, _ in gathered for g in owned) == list(range(p.G))
+    merged = np.zeros_like(ref)
+    for owned, d, tail in gathered:
+        assert tail == 0                              # local segments stay 128-aligned
+        rows = np.isin(p.m_indices, owned)
+        merged[rows] = d[rows]
+        assert (d[~rows] == 0).all()                  # a rank writes only its experts' rows
+    assert np.array_equal(merged, ref)
+
+
+def test_local_contiguous_layout_by_hand():
+    m_idx = np.array([0, 0, -1, -1, 2, -1, 1, 1, 1, -1], np.int32)
+    src, loc = shard.local_contiguous_layout(m_idx, [1, 2], align=4)
+    assert src.tolist() == [6, 7, 8, -1, 4, -1, -1, -1]
+    assert loc.tolist() == [0, 0, 0, -1, 1, -1, -1, -1]
+    src, loc = shard.local_contiguous_layout(m_idx, [], align=4)
+    assert len(src) == 0 and len(loc) == 0
+
+
 @pytest.mark.timeout(300)
 def test_expert_parallel_masked_equals_unsharded():
     results = _run(_rank_masked)
