@@ -253,6 +253,11 @@ int dg_set_tc_util(int percent);
  * order is kept.  enable = 0 launches plainly.  Returns the previous setting. */
 int dg_set_pdl(int enable);
 
+/* The three knobs above take their initial values from the environment when
+ * the library is loaded: DG_NUM_SMS (integer >= 0), DG_TC_UTIL (1..100) and
+ * DG_PDL (0 or 1).  Unset or malformed variables leave the defaults (all SMs,
+ * 100 %, PDL on).  The setters override them at any time. */
+
 /* Forces the tile configuration of the next calls on this host thread:
  * block_n (a built N tile width), ctas (1: 128-row tiles on one SM;
  * 2: 256-row tiles on a pair of SMs; 0: whichever is built, 1 first) and

@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -61,6 +62,25 @@ static int usable_sms(int device_sms) {
 // start its set-up while the previous grid of the stream finishes, and waits
 // (griddepcontrol.wait) before its first global-memory access.
 static std::atomic<int> g_pdl{1};
+
+// Environment defaults of the run-time knobs, read once when the library is
+// loaded: DG_NUM_SMS (as dg_set_num_sms), DG_TC_UTIL (as dg_set_tc_util, a
+// percent) and DG_PDL (as dg_set_pdl, 0 or 1).  A value that is not an
+// integer in the knob's range is ignored.  Calls of the setters override them.
+static int env_int(const char* name, long lo, long hi, int fallback) {
+  const char* v = std::getenv(name);
+  if (v == nullptr || *v == '\0') return fallback;
+  char* end = nullptr;
+  const long x = std::strtol(v, &end, 10);
+  if (*end != '\0' || x < lo || x > hi) return fallback;
+  return static_cast<int>(x);
+}
+static const bool g_env_applied = [] {
+  g_num_sms_override.store(env_int("DG_NUM_SMS", 0, 1 << 20, 0));
+  g_tc_util.store(env_int("DG_TC_UTIL", 1, 100, 100));
+  g_pdl.store(env_int("DG_PDL", 0, 1, 1));
+  return true;
+}();
 
 // One launch attribute set: programmatic stream serialisation when enabled,
 // plus a cluster of `cluster` CTAs along x when cluster > 1.

@@ -148,3 +148,28 @@ def test_binding_argument_helpers_without_gpu():
         dg._out(out.t(), (torch.bfloat16,), (4, 3), "out", out.device)    # not contiguous
     with pytest.raises(ValueError):
         dg._out(out, (torch.bfloat16,), (3, 4), "out", torch.device("meta"))
+
+
+@pytest.mark.parametrize("env,expect_grid,expect_pdl", [
+    ({}, 148, 1),
+    ({"DG_NUM_SMS": "64"}, 64, 1),
+    ({"DG_TC_UTIL": "50"}, 74, 1),
+    ({"DG_TC_UTIL": "abc", "DG_PDL": "0"}, 148, 0),     # malformed value ignored
+    ({"DG_TC_UTIL": "0"}, 148, 1),                     # out of range ignored
+])
+def test_knobs_take_environment_defaults(lib, env, expect_grid, expect_pdl):
+    """DG_NUM_SMS / DG_TC_UTIL / DG_PDL set the knobs' initial values when the
+    library loads (a fresh process per case; no GPU: 148 SMs assumed)."""
+    import os
+    import sys
+
+    code = ("from moe_grouped_gemm_05_b200 import binding as dg; lib = dg.load(); "
+            "print(dg.describe_config('dense', 4096, 7168, 2048).split('/')[-1], lib.dg_set_pdl(1))")
+    clean = {k: v for k, v in os.environ.items() if not k.startswith("DG_")}
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300,
+                         env={**clean, **env, "CUDA_VISIBLE_DEVICES": ""},
+                         cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    assert out.returncode == 0, out.stderr[-2000:]
+    grid, pdl = out.stdout.split()
+    assert int(grid) == expect_grid, out.stdout
+    assert int(pdl) == expect_pdl
