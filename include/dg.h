@@ -259,13 +259,22 @@ int dg_set_pdl(int enable);
  * 100 %, PDL on).  The setters override them at any time. */
 
 /* Forces the tile configuration of the next calls on this host thread:
- * block_n (a built N tile width), ctas (1: 128-row tiles on one SM;
- * 2: 256-row tiles on a pair of SMs; 0: whichever is built, 1 first) and
- * pipes (1: one load/MMA pipeline per CTA; 2: two pipelines taking
- * alternate tiles, each with its own MMA-issuing thread and accumulator,
- * 2-CTA 128- and 224-wide tiles only; 0: either, 1 first).  block_n == 0
- * restores the heuristic.  The contiguous layout only has 1-CTA tiles.
- * Returns DG_OK or DG_ERR_UNSUPPORTED. */
+ * block_n (an N tile width), ctas (1: 128-row tiles on one SM; 2: 256-row
+ * tiles on a pair of SMs; 0: the first built) and pipes (1: one load/MMA
+ * pipeline per CTA; 2: two pipelines, each with its own MMA-issuing thread
+ * and accumulator; 0: the first built).  block_n == 0 restores the heuristic.
+ * Built (block_n, ctas, pipes) triples:
+ *   dense NT and masked : (64|128|224|256, 1, 1), (128|224|256, 2, 1),
+ *                         (128|224, 2, 2) alternate tiles over the pipelines,
+ *                         (64|128, 1, 2) split-K: both pipelines on every tile,
+ *                         each over half of K (used for problems of <= 128 rows)
+ *   contiguous          : (128|224|256, 1, 1), (224, 2, 2)
+ *   FP32 output (_ex)   : (128|224|256, 1, 1)
+ *   NN / TN / TT        : fewer tiles; a forced triple they do not build falls
+ *                         back to the heuristic.
+ * The triple is checked against the dense NT list: DG_OK or DG_ERR_UNSUPPORTED.
+ * A later call of another layout that does not build it returns
+ * DG_ERR_UNSUPPORTED. */
 int dg_set_config(int block_n, int ctas, int pipes);
 
 /* Describes the configuration the heuristic picks for a problem, as
