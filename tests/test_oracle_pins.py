@@ -484,7 +484,12 @@ def test_moe_permute_hand_example():
 def test_moe_permute_invariants():
     rng = np.random.default_rng(19)
     T, topk, G = 500, 3, 7
-    ids = rng.integers(-1, G, size=(T, topk))
+    check_permute_invariants(rng.integers(-1, G, size=(T, topk)), G)
+
+
+def check_permute_invariants(ids, G):
+    """What any correct contiguous-layout permutation of `ids` satisfies."""
+    T, topk = ids.shape
     m, row_of, src, Mt, bad = oracle.fp8_gemm.moe_permute(ids, G)
     assert Mt % 128 == 0 and len(m) == Mt and bad == 0
     assert Mt <= oracle.fp8_gemm.moe_permute_capacity(T, topk, G)

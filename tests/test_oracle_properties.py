@@ -97,3 +97,42 @@ def test_bf16_rounding_near_midpoints(bits, negative, side, depth):
     xf = float(x)
     assert Fraction(xf) == x                                  # exactly representable in float64
     assert int(oracle.bf16_bits_from_f64(np.array([xf]))[0]) == _frac_to_bf16_bits(x)
+
+
+@SETTINGS
+@given(st.integers(1, 4), st.integers(1, 3), st.integers(0, 2 ** 32 - 1), st.integers(-30, 30))
+def test_quantize_scale_is_minimal_and_codes_match_torch_cast(rows, groups, seed, log_mag):
+    """Per 128-wide group: the scale s is the smallest power of two with
+    amax / s <= 448 (1 for an all-zero group), and the codes are PyTorch's own
+    float8_e4m3fn cast of x / s."""
+    import torch
+
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, 128 * groups)) * np.exp2(log_mag + rng.integers(-8, 9, size=(rows, 1)))
+    x = x.astype(np.float32).astype(np.float64)
+    if rows > 1:
+        x[1, :128] = 0.0                                        # an all-zero group
+    codes, words = oracle.fp8_gemm.quantize_fp8_1x128(x)
+    e = oracle.unpack_sf_ue8m0(words[None], rows, groups)[0].astype(np.int64)
+    for r in range(rows):
+        for g in range(groups):
+            grp = x[r, 128 * g:128 * (g + 1)]
+            amax = Fraction(float(np.abs(grp).max()))
+            s = Fraction(2) ** int(e[r, g] - 127)
+            if amax == 0:
+                assert s == 1
+            else:
+                assert amax / s <= 448 and amax / (s / 2) > 448
+            ref = torch.from_numpy((grp / float(s)).astype(np.float32)).to(torch.float8_e4m3fn)
+            assert np.array_equal(codes[r, 128 * g:128 * (g + 1)], ref.view(torch.uint8).numpy())
+
+
+@SETTINGS
+@given(st.integers(1, 300), st.integers(1, 4), st.integers(1, 40), st.floats(0.0, 0.5), st.integers(0, 2 ** 32 - 1))
+def test_moe_permute_invariants_random(T, topk, G, drop, seed):
+    from test_oracle_pins import check_permute_invariants
+
+    rng = np.random.default_rng(seed)
+    ids = rng.integers(0, G, size=(T, topk))
+    ids[rng.random((T, topk)) < drop] = -1
+    check_permute_invariants(ids, G)
