@@ -173,3 +173,68 @@ def test_knobs_take_environment_defaults(lib, env, expect_grid, expect_pdl):
     grid, pdl = out.stdout.split()
     assert int(grid) == expect_grid, out.stdout
     assert int(pdl) == expect_pdl
+
+
+def test_every_other_entry_point_rejects_bad_arguments_on_the_host(lib):
+    """Argument errors come back as status codes before any device query or
+    launch, for the entry points not covered above (runs without a GPU)."""
+    odd4 = P(0x10004)   # 4-byte but not 16-byte aligned
+    for name in ("dg_fp8_gemm_nn", "dg_fp8_gemm_tn", "dg_fp8_gemm_tt"):
+        f = getattr(lib, name)
+        assert f(P(0), GOOD, GOOD, GOOD, GOOD, 128, 256, 256, None) == -1, name
+        assert f(GOOD, GOOD, GOOD, GOOD, P(0x10008), 128, 256, 256, None) == -3, name
+        assert f(GOOD, GOOD, GOOD, GOOD, GOOD, 128, 256, 100, None) == -2, name
+        assert f(GOOD, GOOD, GOOD, GOOD, GOOD, 128, 200, 256, None) == -2, name
+        assert f(GOOD, GOOD, GOOD, GOOD, GOOD, -1, 256, 256, None) == -2, name
+        assert f(GOOD, GOOD, GOOD, GOOD, GOOD, 0, 256, 256, None) == 0, name
+    # A stored [K][M] (TN, TT): its rows are M bytes, which must be a multiple of 16
+    assert lib.dg_fp8_gemm_tn(GOOD, GOOD, GOOD, GOOD, GOOD, 120, 256, 256, None) == -2
+    assert lib.dg_fp8_gemm_tt(GOOD, GOOD, GOOD, GOOD, GOOD, 120, 256, 256, None) == -2
+
+    ex = lib.dg_fp8_gemm_nt_ex
+    assert ex(GOOD, GOOD, GOOD, GOOD, None, GOOD, 128, 256, 256, 64, 0, None) == -4   # granularity 1 or 128
+    assert ex(GOOD, GOOD, GOOD, GOOD, None, GOOD, 128, 256, 256, 128, 2, None) == -4  # d_is_fp32 0 or 1
+    assert ex(GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 128, 256, 256, 128, 0, None) == -4  # C needs an FP32 d
+    assert ex(GOOD, GOOD, GOOD, GOOD, P(0x10008), GOOD, 128, 256, 256, 128, 1, None) == -3
+    assert ex(GOOD, GOOD, GOOD, GOOD, None, GOOD, 0, 256, 256, 1, 1, None) == 0
+
+    # fp32 A scales need 4-byte alignment only; packed words need 16
+    f32 = lib.dg_fp8_gemm_nt_fp32sfa
+    assert f32(GOOD, odd4, GOOD, GOOD, GOOD, 0, 256, 256, None) == 0
+    assert f32(GOOD, P(0x10002), GOOD, GOOD, GOOD, 0, 256, 256, None) == -3
+    assert lib.dg_fp8_gemm_nt(GOOD, odd4, GOOD, GOOD, GOOD, 0, 256, 256, None) == -3
+    cf = lib.dg_m_grouped_fp8_gemm_nt_contiguous_fp32sfa
+    assert cf(GOOD, odd4, GOOD, GOOD, GOOD, GOOD, 0, 256, 256, 4, None) == 0
+    assert cf(GOOD, odd4, GOOD, GOOD, GOOD, GOOD, 200, 256, 256, 4, None) == -2
+    mf = lib.dg_m_grouped_fp8_gemm_nt_masked_fp32sfa
+    assert mf(GOOD, odd4, GOOD, GOOD, GOOD, P(0), 4, 256, 256, 256, None) == -1
+    assert mf(GOOD, odd4, GOOD, GOOD, GOOD, GOOD, 4, 0, 256, 256, None) == 0
+
+    q = lib.dg_quantize_fp8_1x128
+    assert q(P(0), 0, GOOD, GOOD, 1, 128, 256, None) == -1
+    assert q(GOOD, 2, GOOD, GOOD, 1, 128, 256, None) == -4                 # dtype code 0 (bf16) or 1 (fp32)
+    assert q(GOOD, 0, odd4, GOOD, 1, 128, 256, None) == -3
+    assert q(GOOD, 0, GOOD, GOOD, 1, 128, 200, None) == -2
+    assert q(GOOD, 0, GOOD, GOOD, -1, 128, 256, None) == -2
+    assert q(GOOD, 0, GOOD, GOOD, 0, 128, 256, None) == 0                  # empty batch: nothing to do
+
+    cap = lib.dg_moe_permute_capacity
+    assert cap(100, 2, 4) == (200 + 127 * 4 + 127) // 128 * 128
+    assert cap(-1, 2, 4) == -2 and cap(10, 0, 4) == -2 and cap(10, 2, 0) == -2
+    perm = lib.dg_moe_permute
+    c = cap(100, 2, 4)
+    args = lambda **kw: [kw.get("ids", GOOD), kw.get("T", 100), kw.get("topk", 2), kw.get("G", 4), kw.get("q", GOOD),
+                         GOOD, kw.get("K", 256), GOOD, GOOD, GOOD, GOOD, GOOD, kw.get("M_cap", c), None]
+    assert perm(*args(ids=P(0))) == -1
+    assert perm(*args(q=odd4)) == -3
+    assert perm(*args(G=1025)) == -2                                       # at most 1024 experts
+    assert perm(*args(K=100)) == -2
+    assert perm(*args(M_cap=c - 128)) == -2                                # below the capacity
+    assert perm(*args(M_cap=c + 64)) == -2                                 # not a multiple of 128
+
+    comb = lib.dg_moe_unpermute_combine
+    assert comb(P(0), GOOD, None, 10, 2, 256, GOOD, None) == -1
+    assert comb(GOOD, GOOD, None, 10, 2, 256, odd4, None) == -3
+    assert comb(GOOD, GOOD, None, 10, 0, 256, GOOD, None) == -2
+    assert comb(GOOD, GOOD, None, 10, 2, 200, GOOD, None) == -2
+    assert comb(GOOD, GOOD, None, 0, 2, 256, GOOD, None) == 0              # no tokens: nothing to do
