@@ -238,3 +238,33 @@ def test_every_other_entry_point_rejects_bad_arguments_on_the_host(lib):
     assert comb(GOOD, GOOD, None, 10, 0, 256, GOOD, None) == -2
     assert comb(GOOD, GOOD, None, 10, 2, 200, GOOD, None) == -2
     assert comb(GOOD, GOOD, None, 0, 2, 256, GOOD, None) == 0              # no tokens: nothing to do
+
+
+def test_last_error_and_forced_config_are_per_thread(lib):
+    """dg_get_last_error() and dg_set_config() are per host thread: one
+    thread's failure text and forced tiles do not leak into another's."""
+    import threading
+
+    from moe_grouped_gemm_05_b200 import binding as dg
+
+    barrier = threading.Barrier(2)
+    seen = {}
+
+    def worker(name, K, force):
+        if force:
+            assert lib.dg_set_config(128, 1, 1) == 0
+        assert _dense(lib, K=K) == -2
+        barrier.wait()                    # both threads have failed before either reads its text
+        seen[name] = (lib.dg_get_last_error().decode(), dg.describe_config("dense", 4096, 7168, 2048))
+        barrier.wait()
+        lib.dg_set_config(0, 0, 0)
+
+    threads = [threading.Thread(target=worker, args=("a", 100, True)),
+               threading.Thread(target=worker, args=("b", 300, False))]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=60)
+    assert "K=100" in seen["a"][0] and "K=300" in seen["b"][0]
+    assert seen["a"][1].startswith("128x128x6/")                      # forced on thread a only
+    assert seen["b"][1] == "256x224x6(2cta)(2pipe)/148"              # thread b keeps the heuristic
