@@ -122,7 +122,7 @@ class ClockSampler:
                 self._handle = pynvml.nvmlDeviceGetHandleByIndex(torch_dev)
             self._nvml = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM)
-        except Exception:  # noqa: BLE001 - clocks are best effort off the GPU machine
+        except Exception:  # noqa: BLE001 - clock sampling is best effort (NVML may be absent)
             self._handle = None
 
     def _run(self):

@@ -1,7 +1,7 @@
 """GPU parity of the extended dense entry point: the 1D1D recipe (per-row B
 scales), FP32 output and accumulation into an FP32 C.
 
-FP32 outputs keep the task's row term: |x - y| <= ulp_f32(y) + 2^-10 * max|y[row]|,
+FP32 outputs keep the BF16 tolerance's row term: |x - y| <= ulp_f32(y) + 2^-10 * max|y[row]|,
 with the normalised difference < 1e-4; integer-valued problems are bit exact."""
 import numpy as np
 import pytest
