@@ -8,11 +8,20 @@ on them (--fused-pack: the GEMM reads the fp32 scales and its scale-producer
 warp packs them, one launch per step).  Weight scales are packed once, as a
 deployment would.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--workloads all|none|a,b]
+                    [--impl ours|reference]
 
-Prints ONE JSON line on rank 0.  With N > 1 (torchrun, one process per GPU)
-every rank runs its own independent problem (weak scaling, no collective on
-the data path); the time is the max over ranks.
+Prints ONE JSON line on rank 0.  Its top level is the headline workload,
+the largest of the five (the contiguous M-grouped GEMM, 8 experts, 32768
+Zipf-routed rows, N=4096, K=7168); with one GPU the same line carries a
+``workloads`` object with every workload measured in the same run (kernel
+configuration, time, TFLOPS, roofline fraction and the CPU oracle's rate).
+
+With N > 1 (torchrun, one process per GPU) the headline problem is split
+across the ranks along N in whole 128-column blocks (each rank holds A, its
+slice of every expert's weights and its columns of D; ``--shard experts``
+splits the experts instead): strong scaling, no collective on the data path,
+time = max over ranks.
 """
 from __future__ import annotations
 
@@ -31,7 +40,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "FP8 block-scaled GEMM TFLOPS (dense/grouped/masked) and % of B200 roofline"
-DEFAULT_WORKLOAD = "dense_4096x7168x2048"
+DEFAULT_WORKLOAD = "contiguous_8x4096x7168_zipf1.1"
+ALL_WORKLOADS = ("dense_128x512x512", "dense_4096x7168x2048", "dense_64x7168x2048",
+                 "contiguous_8x4096x7168_zipf1.1", "masked_16x256x7168x2048", "dense_8192x8192x8192_outliers")
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -42,13 +53,20 @@ REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_c
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, help="the headline workload (top level of the line)")
+    ap.add_argument("--workloads", default="all",
+                    help="workloads measured into the line's 'workloads' object at N=1: all, none or a comma list")
+    ap.add_argument("--shard", choices=["n", "experts"], default="n",
+                    help="N > 1: split N across ranks (default) or, for grouped workloads, the experts")
+    ap.add_argument("--min-window-ms", type=float, default=200.0,
+                    help="each timing is repeated (K-step graph replays) until this much device time is covered")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the headline's oracle sample")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end loop (0 = min(steps, 100))")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end loop (profiling runs)")
     ap.add_argument("--eager", action="store_true", help="time host-issued launches instead of a CUDA graph")
     ap.add_argument("--fused-pack", action="store_true",
                     help="let the GEMM read A's fp32 scales and pack them itself instead of a packing launch")
@@ -330,38 +348,57 @@ def run_reference(args):
     return 0
 
 
-def run_ours(args):
-    import torch
-    import torch.distributed as dist
+def shard_problem(p, world: int, rank: int, how: str):
+    """This rank's share of problem `p` (strong scaling, no exchange step).
 
-    from moe_grouped_gemm_05_b200 import binding as dg
-    from moe_grouped_gemm_05_b200 import shard, synth
+    "n": columns [n0, n1) of every expert in whole 128-column blocks (A and
+    the routing are replicated); "experts" (grouped problems): the experts
+    ``shard.partition_experts`` gives this rank, re-laid out with
+    ``shard.local_contiguous_layout`` (contiguous) or selected (masked)."""
+    import dataclasses
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world != args.gpus and world > 1:
-        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
+    from moe_grouped_gemm_05_b200 import shard
 
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    if world == 1:
+        return p
+    if how == "experts" and p.kind != "dense":
+        if p.kind == "contiguous":
+            counts = np.bincount(p.m_indices[p.m_indices >= 0], minlength=p.G)
+            owned = shard.partition_experts(counts, world)[rank]
+            src, loc = shard.local_contiguous_layout(p.m_indices, owned)
+            keep = src >= 0
+            a = np.zeros((len(src), p.K), np.uint8)
+            a[keep] = p.a[src[keep]]
+            sfa = np.ones((len(src), p.sfa.shape[1]), np.float32)
+            sfa[keep] = p.sfa[src[keep]]
+            return dataclasses.replace(p, a=a, sfa=sfa, b=p.b[owned], sfb=p.sfb[owned], M=len(src), G=len(owned),
+                                       m_indices=loc.astype(np.int32), name=f"{p.name}_experts{rank}of{world}")
+        owned = shard.partition_experts(p.masked_m, world)[rank]
+        return dataclasses.replace(p, a=p.a[owned], sfa=p.sfa[owned], b=p.b[owned], sfb=p.sfb[owned], G=len(owned),
+                                   masked_m=p.masked_m[owned], name=f"{p.name}_experts{rank}of{world}")
+    n0, n1 = shard.split_n(p.N, world, rank)
+    b = np.ascontiguousarray(p.b[..., n0:n1, :])
+    sfb = np.ascontiguousarray(p.sfb[..., n0 // 128:(n1 + 127) // 128, :])
+    return dataclasses.replace(p, b=b, sfb=sfb, N=n1 - n0, name=f"{p.name}_n{n0}-{n1}")
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
 
-    lib = dg.load()
-    # every rank runs its own copy of the problem: independent units, weak scaling
-    maker = synth.WORKLOADS[args.workload]
-    p = maker()
+class Measured(dict):
+    pass
+
+
+def measure(p, dg, lib, torch, args, dev, local, barrier):
+    """Times K steps (pack + GEMM) and K GEMM launches of problem `p`.
+
+    Each timing is a CUDA-graph replay of the K launches (or host-issued
+    launches with --eager), bracketed by events on the launching stream;
+    replays are repeated until --min-window-ms of device time is covered,
+    and the median replay is reported.  Inputs rotate over enough device
+    copies that their total exceeds 2x L2.  NVML clocks are sampled during
+    the replays."""
     sets, per_set = make_device_sets(p, dg, torch, dev)
     nsets = len(sets)
-    stream = torch.cuda.current_stream()
-
     fused = args.fused_pack
+    K = args.steps
 
     def step(i):
         s = sets[i % nsets]
@@ -369,75 +406,110 @@ def run_ours(args):
             pack_call(dg, lib, s, torch)
         gemm_call(p, dg, s, fp32_sfa=fused)
 
+    def gemm_only(i):
+        gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
+
     for i in range(args.warmup):
         step(i)
     torch.cuda.synchronize()
-    assert dg.get_device_error() == 0, "device error word set during warm-up"
+    assert dg.get_device_error() == 0, f"{p.name}: device error word set during warm-up"
     kernel_desc = dg.describe_config(p.kind, p.M, p.N, p.K, p.G)
 
-    # The K timed steps are captured once as a CUDA graph and replayed, so the
-    # device runs them back to back without host launch gaps (--eager times
-    # host-issued launches instead).  A second graph holds the K GEMM launches
-    # alone and gives the kernel's own average duration.
-    cap = torch.cuda.Stream()
-    step_graph = gemm_graph = None
+    graphs = {}
     if not args.eager:
+        cap = torch.cuda.Stream()
         with torch.cuda.stream(cap):
             cap.wait_stream(torch.cuda.current_stream())
-            step_graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(step_graph, stream=cap):
-                for i in range(args.steps):
-                    step(i)
-            gemm_graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gemm_graph, stream=cap):
-                for i in range(args.steps):
-                    gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
+            for name, fn in (("step", step), ("gemm", gemm_only)):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=cap):
+                    for i in range(K):
+                        fn(i)
+                graphs[name] = g
         torch.cuda.synchronize()
-        step_graph.replay()  # upload + untimed pass
-        gemm_graph.replay()
+        for g in graphs.values():  # upload + untimed pass
+            g.replay()
         torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local).start()
-    barrier()
-    torch.cuda.synchronize()
-    start.record(stream)
-    if step_graph is not None:
-        step_graph.replay()
-    else:
-        for i in range(args.steps):
-            step(i)
-    end.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    elapsed_ms = start.elapsed_time(end)
-    # kernel-only timing on the same stream, right after the timed region
-    g0 = torch.cuda.Event(enable_timing=True)
-    g1 = torch.cuda.Event(enable_timing=True)
-    g0.record(stream)
-    if gemm_graph is not None:
-        gemm_graph.replay()
-    else:
-        for i in range(args.steps):
-            gemm_call(p, dg, sets[i % nsets], fp32_sfa=fused)
-    g1.record(stream)
-    torch.cuda.synchronize()
-    sampler.stop()
-    gemm_avg_ms = g0.elapsed_time(g1) / args.steps
-    elapsed_ms = shard.max_over_ranks(elapsed_ms)
-    gemm_avg_ms = shard.max_over_ranks(gemm_avg_ms)
-    err = dg.get_device_error()
 
-    # End to end through the public API: every step copies its inputs from
-    # pinned host memory, packs + multiplies, and copies D back to pinned host
-    # memory.  When a step moves at least 8 MB, consecutive steps overlap on
-    # three streams over two device buffer sets (H2D of step i+1 and D2H of
-    # step i-1 run beside step i's GEMM), as a serving loop would; smaller
-    # steps, bound by copy-launch latency, run on one stream.  The time runs
-    # from the first copy in to the last copy out.
+    def timed(name, fn):
+        """Median device time (ms) of one replay of K launches, and the replay count."""
+        def once():
+            if name in graphs:
+                graphs[name].replay()
+            else:
+                for i in range(K):
+                    fn(i)
+        ev = []
+        total_ms, reps = 0.0, 0
+        barrier()
+        torch.cuda.synchronize()
+        while reps < 3 or (total_ms < args.min_window_ms and reps < 5000):
+            batch = max(1, min(64, reps + 1))
+            pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(batch)]
+            for a, b in pairs:
+                a.record(stream)
+                once()
+                b.record(stream)
+            torch.cuda.synchronize()
+            for a, b in pairs:
+                ev.append(a.elapsed_time(b))
+            total_ms = sum(ev)
+            reps = len(ev)
+        barrier()
+        return statistics.median(ev), reps
+
+    sampler = ClockSampler(local).start()
+    step_ms, step_reps = timed("step", step)
+    gemm_ms, gemm_reps = timed("gemm", gemm_only)
+    sampler.stop()
+    err = dg.get_device_error()
+    m = Measured(p=p, sets=sets, per_set=per_set, nsets=nsets, kernel_desc=kernel_desc,
+                 step_ms=step_ms / K, gemm_ms=gemm_ms / K, replays=step_reps, gemm_replays=gemm_reps,
+                 window_ms=step_ms * step_reps, clocks=sampler.summary(), device_error=err)
+    del graphs
+    return m
+
+
+def roofline_of(p, gemm_ms, clocks, window_ms, workload_key, kernel_desc):
+    peaks, peak_src = load_peaks()
+    bound = bound_of(p)
+    # The sustained peak was measured under the power cap: use it when the timed
+    # windows were long or the clock sampler saw the cap; the burst peak otherwise.
+    power_capped = "sw_power_cap" in clocks.get("reasons", [])
+    long_region = window_ms > 500.0 or power_capped
+    if bound == "tensor":
+        bf16 = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+        peak = 2.0 * bf16  # FP8 dense = 2 x BF16 dense (nominal ratio)
+        achieved = p.flops / (gemm_ms * 1e-3) / 1e12
+        unit = "TFLOP/s"
+        note = (f"{'sustained' if long_region else 'burst'} bf16 x2 ({peak_src} peaks)"
+                + ("; power cap active during the timed region" if power_capped else ""))
+    else:
+        peak = peaks.get("hbm_gbs")
+        achieved = algorithmic_bytes(p) / (gemm_ms * 1e-3) / 1e9
+        unit = "GB/s"
+        note = f"copy bandwidth ({peak_src} peaks)"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak if peak else None, "traffic": recorded_traffic(workload_key, kernel_desc),
+            "traffic_note": ("DRAM read + write bytes of one launch from a committed ncu capture of this kernel "
+                             "code and configuration; D rows still in L2 when the kernel ends are not counted"),
+            "peak_source": note, "kernel": "fp8_gemm_kernel", "kernel_ms_avg": gemm_ms,
+            "algorithmic": (f"{p.flops:.4g} FLOP" if bound == "tensor" else f"{algorithmic_bytes(p):.4g} B")
+            + " per launch"}
+
+
+def e2e_loop(p, m, dg, lib, torch, args, barrier):
+    """End to end through the public API: every step copies its inputs from
+    pinned host memory, packs + multiplies, and copies D back to pinned host
+    memory.  When a step moves at least 8 MB, consecutive steps overlap on
+    three streams over two device buffer sets (H2D of step i+1 and D2H of
+    step i-1 run beside step i's GEMM), as a serving loop would; smaller
+    steps, bound by copy-launch latency, run on one stream.  The time runs
+    from the first copy in to the last copy out."""
+    sets, fused = m["sets"], args.fused_pack
     e2e_steps = args.e2e_steps or min(args.steps, 100)
-    if nsets > 1:
+    if len(sets) > 1:
         bufs = [sets[0], sets[1]]
     else:  # one set is already > 2x L2: a second one for A, its scales and D (B shared)
         s1 = dict(sets[0])
@@ -503,57 +575,113 @@ def run_ours(args):
     e1.record(first)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = shard.max_over_ranks(e0.elapsed_time(e1))
+    return {"ms": e0.elapsed_time(e1), "steps": e2e_steps, "h2d": h2d, "d2h": d2h, "overlap": overlap}
 
-    flops = p.flops
-    value = world * flops * args.steps / (elapsed_ms * 1e-3) / 1e12
-    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
-    peaks, peak_src = load_peaks()
-    bound = bound_of(p)
-    # The sustained peak was measured under the power cap: use it when the timed
-    # region was long or the clock sampler saw the cap; the burst peak otherwise.
-    clocks = sampler.summary()
-    power_capped = "sw_power_cap" in clocks.get("reasons", [])
-    long_region = elapsed_ms > 500.0 or power_capped
-    if bound == "tensor":
-        bf16 = peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
-        peak = 2.0 * bf16  # FP8 dense = 2 x BF16 dense (nominal ratio)
-        achieved = flops / (gemm_avg_ms * 1e-3) / 1e12
-        unit = "TFLOP/s"
-        peak_note = (f"{'sustained' if long_region else 'burst'} bf16 x2 ({peak_src})"
-                     + ("; power cap active during the timed region" if power_capped else ""))
-    else:
-        peak = peaks.get("hbm_gbs")
-        achieved = algorithmic_bytes(p) / (gemm_avg_ms * 1e-3) / 1e9
-        unit = "GB/s"
-        peak_note = f"copy bandwidth ({peak_src})"
-    traffic = recorded_traffic(args.workload, kernel_desc)
 
+def cpu_baseline_of(p, seconds):
+    smp = OracleSample(p)
+    rows = smp.calibrate(seconds)
+    return smp.info(rows, smp.run(rows))
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from moe_grouped_gemm_05_b200 import binding as dg
+    from moe_grouped_gemm_05_b200 import shard, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    lib = dg.load()
+    full = synth.WORKLOADS[args.workload]()
+    p = shard_problem(full, world, rank, args.shard)
+    m = measure(p, dg, lib, torch, args, dev, local, barrier)
+    e2e = None if args.no_e2e else e2e_loop(p, m, dg, lib, torch, args, barrier)
+    m["sets"] = None
+    torch.cuda.empty_cache()
+
+    # max over ranks of every time; the work is the whole (unsharded) problem's
+    step_ms = shard.max_over_ranks(m["step_ms"])
+    gemm_ms = shard.max_over_ranks(m["gemm_ms"])
+    e2e_ms = shard.max_over_ranks(e2e["ms"]) if e2e else None
+    flops = full.flops
+    value = flops / (step_ms * 1e-3) / 1e12
+    # roofline of this rank's kernel on this rank's share (rank 0 reports it)
+    roof = roofline_of(p, m["gemm_ms"], m["clocks"], m["window_ms"], args.workload if world == 1 else p.name,
+                       m["kernel_desc"])
+    clocks = m["clocks"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3", "data": "synthetic",
-        "config": {"workload": args.workload, "kind": p.kind, "M": p.M, "N": p.N, "K": p.K, "G": p.G,
-                   "valid_rows": p.valid_rows, "kernel_config": kernel_desc,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
+        "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "kind": full.kind, "M": full.M, "N": full.N, "K": full.K, "G": full.G,
+                   "valid_rows": full.valid_rows, "kernel_config": m["kernel_desc"],
+                   "parallelism": (f"{world} ranks, " + ("N split in 128-column blocks" if args.shard == "n"
+                                                         or full.kind == "dense" else "experts split")
+                                   if world > 1 else "one GPU"),
                    "step": ("GEMM reading A's fp32 scales, packed to UE8M0 in its scale-producer warp"
-                            if fused else "pack activation scales (fp32 -> UE8M0 int32) + GEMM"),
-                   "timing": "eager launches" if args.eager else "CUDA-graph replay of the K steps",
-                   "l2": f"inputs rotate over {nsets} device copies ({nsets * per_set / 1e6:.0f} MB > 2x L2)"},
-        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                     "frac": achieved / peak if peak else None, "traffic": traffic, "peak_source": peak_note,
-                     "kernel": "fp8_gemm_kernel", "kernel_ms_avg": gemm_avg_ms},
-        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": e2e_steps,
-                "overlap": ("H2D / compute / D2H of consecutive steps on three streams" if overlap
-                            else "none: one stream (less than 8 MB of copies per step)")},
-        "gpu_launches": (1 if fused else 2) * args.steps,
+                            if args.fused_pack else "pack activation scales (fp32 -> UE8M0 int32) + GEMM"),
+                   "timing": (("eager launches" if args.eager else "CUDA-graph replay of the K steps")
+                              + f"; median of {m['replays']} replays ({m['window_ms']:.0f} ms of device time)"),
+                   "l2": (f"inputs rotate over {m['nsets']} device copies "
+                          f"({m['nsets'] * m['per_set'] / 1e6:.0f} MB > 2x L2)")},
+        "roofline": roof,
+        "gpu_launches": (1 if args.fused_pack else 2) * args.steps,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-        "device_error": err,
+        "device_error": m["device_error"],
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        smp = OracleSample(p)
-        rows = smp.calibrate(args.cpu_seconds)
-        line["cpu_baseline"] = smp.info(rows, smp.run(rows))
+    if e2e:
+        line["e2e"] = {"value": flops * e2e["steps"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
+                       "overlap": ("H2D / compute / D2H of consecutive steps on three streams" if e2e["overlap"]
+                                   else "none: one stream (less than 8 MB of copies per step)")}
+
+    # every workload in the same run (one GPU): kernel configuration, time, rate, roofline, CPU oracle
+    names = []
+    if world == 1 and args.workloads != "none":
+        names = list(ALL_WORKLOADS) if args.workloads == "all" else args.workloads.split(",")
+    if names:
+        line["workloads"] = {}
+    for name in names:
+        if name == args.workload:
+            q, mq = full, m
+        else:
+            q = synth.WORKLOADS[name]()
+            mq = measure(q, dg, lib, torch, args, dev, local, barrier)
+            mq["sets"] = None
+            torch.cuda.empty_cache()
+        entry = {"kind": q.kind, "M": q.M, "N": q.N, "K": q.K, "G": q.G, "valid_rows": q.valid_rows,
+                 "kernel_config": mq["kernel_desc"], "ms_per_step": mq["step_ms"], "kernel_ms_avg": mq["gemm_ms"],
+                 "value": q.flops / (mq["step_ms"] * 1e-3) / 1e12, "unit": "TFLOPS",
+                 "kernel_tflops": q.flops / (mq["gemm_ms"] * 1e-3) / 1e12,
+                 "roofline": roofline_of(q, mq["gemm_ms"], mq["clocks"], mq["window_ms"], name, mq["kernel_desc"]),
+                 "replays": mq["replays"], "window_ms": mq["window_ms"],
+                 "clocks": {k: mq["clocks"][k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+                 "device_error": mq["device_error"]}
+        if not args.no_cpu_baseline:
+            secs = args.cpu_seconds if name == args.workload else max(1.0, args.cpu_seconds / 2)
+            entry["cpu_baseline"] = cpu_baseline_of(q, secs)
+            if name == args.workload:
+                line["cpu_baseline"] = entry["cpu_baseline"]
+        line["workloads"][name] = entry
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and "cpu_baseline" not in line:
+        line["cpu_baseline"] = cpu_baseline_of(full, args.cpu_seconds)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

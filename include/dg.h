@@ -229,9 +229,23 @@ int dg_get_mk_alignment_for_contiguous_layout(void);
 /* Number of int32 words of one packed scale matrix: ceil(kb/4) * align4(mn). */
 int64_t dg_packed_sf_words(int mn, int kb);
 
-/* Synchronises `stream`, returns the current device's error word in *err
- * (0 = none, else DG_DEVERR_* bits) and clears it. */
+/* Returns the current device's error word in *err (0 = none, else DG_DEVERR_*
+ * bits) and clears it, in one atomic step on the device that is ordered after
+ * the earlier work of `stream`; then synchronises `stream`.  Bits that
+ * kernels on other streams set meanwhile stay in the word for the next read.
+ * (Failure contract of the nightvoyager.top report's "解法哲学": errors are
+ * reported, not trapped.) */
 int dg_get_device_error(void* stream, int* err);
+
+/* Time limit of each pipeline wait inside the GEMM kernels, in nanoseconds,
+ * for every later call in this process (default 2e9, i.e. 2 s).  A wait that
+ * runs out sets DG_DEVERR_TIMEOUT; every role of that CTA then stops
+ * issuing, waits (with the 2 s limit, whatever this setting) for its own
+ * copies and tensor-core operations in flight, frees its tensor memory and
+ * exits, so the context stays usable and the output is incomplete.  A short
+ * limit (0 included) makes an ordinary call give up: it exists to exercise
+ * that path.  Returns the previous limit. */
+uint64_t dg_set_wait_limit_ns(uint64_t ns);
 
 /* Persistent-grid size (the ssnai.com analysis' set_num_sms knob).
  * n <= 0 restores "all SMs".  Returns the previous setting. */
@@ -270,11 +284,10 @@ int dg_set_pdl(int enable);
  *                         each over half of K (used for problems of <= 128 rows)
  *   contiguous          : (128|224|256, 1, 1), (224, 2, 2)
  *   FP32 output (_ex)   : (128|224|256, 1, 1)
- *   NN / TN / TT        : fewer tiles; a forced triple they do not build falls
- *                         back to the heuristic.
- * The triple is checked against the dense NT list: DG_OK or DG_ERR_UNSUPPORTED.
- * A later call of another layout that does not build it returns
- * DG_ERR_UNSUPPORTED. */
+ *   NN / TN / TT        : fewer tiles.
+ * The triple must be built for at least one entry point (else
+ * DG_ERR_UNSUPPORTED).  An entry point that does not build it keeps the
+ * heuristic's choice. */
 int dg_set_config(int block_n, int ctas, int pipes);
 
 /* Describes the configuration the heuristic picks for a problem, as

@@ -69,6 +69,8 @@ def load() -> ctypes.CDLL:
     lib.dg_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int)]
     lib.dg_set_num_sms.argtypes = [i]
     lib.dg_set_pdl.argtypes = [i]
+    lib.dg_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.dg_set_wait_limit_ns.restype = ctypes.c_uint64
     lib.dg_set_tc_util.argtypes = [i]
     lib.dg_get_num_sms.argtypes = []
     lib.dg_set_config.argtypes = [i, i, i]
@@ -388,10 +390,17 @@ def moe_unpermute_combine(d_perm: torch.Tensor, row_of: torch.Tensor, weights=No
 
 
 def get_device_error() -> int:
-    """Synchronises the current stream, returns and clears the device error word."""
+    """Returns and clears the device error word (atomically, after the current stream's work)."""
     v = ctypes.c_int(0)
     _check(load().dg_get_device_error(_stream(), ctypes.byref(v)))
     return v.value
+
+
+def set_wait_limit_ns(ns: int) -> int:
+    """Sets the time limit of each pipeline wait in the GEMM kernels; returns the previous one."""
+    if ns < 0:
+        raise ValueError("the wait limit is a non-negative number of nanoseconds")
+    return int(load().dg_set_wait_limit_ns(ns))
 
 
 def set_num_sms(n: int) -> int:

@@ -62,6 +62,8 @@ static int usable_sms(int device_sms) {
 // start its set-up while the previous grid of the stream finishes, and waits
 // (griddepcontrol.wait) before its first global-memory access.
 static std::atomic<int> g_pdl{1};
+// Limit of every main-loop pipeline wait inside the GEMM kernels, in ns.
+static std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
 
 // Environment defaults of the run-time knobs, read once when the library is
 // loaded: DG_NUM_SMS (as dg_set_num_sms), DG_TC_UTIL (as dg_set_tc_util, a
@@ -309,9 +311,10 @@ static double config_rate(const Config& c) {
 
 template <int MODE>
 static const Config* choose_config(long long rows_est, int N, int K, int sms, int groups = 1) {
+  // A forced tile applies to the entry points that have it built; the others
+  // keep the heuristic (each layout and output type builds its own set).
   if (t_force_bn) {
     if (const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes)) return f;
-    if (MODE < MODE_DENSE_MN) return nullptr;  // layouts build fewer tiles: fall back to the heuristic
   }
   (void)K;
   int n = 0;
@@ -378,8 +381,9 @@ static int max_active_pairs(const Config* cfg, int sms) {
 }
 
 template <int MODE>
-static int launch(const Config* cfg, int grid, const CUtensorMap* maps, const GemmArgs& args,
+static int launch(const Config* cfg, int grid, const CUtensorMap* maps, GemmArgs args,
                   cudaStream_t stream) {
+  args.wait_limit_ns = g_wait_limit_ns.load(std::memory_order_relaxed);
   // The shared-memory opt-in is a per-device function attribute: set it once
   // per (device, configuration).
   constexpr int kMaxDevices = 64, kMaxConfigs = 32;
@@ -565,6 +569,14 @@ __global__ void pack_sf_ue8m0_kernel(const float* __restrict__ sf, uint32_t* __r
   }
 }
 
+// The error word as last taken by take_error_kernel (one per device).
+__device__ int g_dg_error_taken = 0;
+
+// Reads and clears the error word in one atomic step, ordered after the
+// stream's earlier work; bits set meanwhile by kernels on other streams stay
+// in the word for the next read.
+__global__ void take_error_kernel() { g_dg_error_taken = atomicExch(&g_dg_error, 0); }
+
 }  // namespace dg
 
 using namespace dg;
@@ -639,7 +651,10 @@ int dg_set_config(int block_n, int ctas, int pipes) {
   }
   if (ctas < 0 || ctas > 2) return fail(DG_ERR_UNSUPPORTED, "ctas=%d must be 0, 1 or 2", ctas);
   if (pipes < 0 || pipes > 2) return fail(DG_ERR_UNSUPPORTED, "pipes=%d must be 0, 1 or 2", pipes);
-  if (!find_config<MODE_DENSE>(block_n, ctas, pipes))
+  if (!find_config<MODE_DENSE>(block_n, ctas, pipes) && !find_config<MODE_CONTIG>(block_n, ctas, pipes) &&
+      !find_config<MODE_MASKED>(block_n, ctas, pipes) && !find_config<MODE_DENSE_F32>(block_n, ctas, pipes) &&
+      !find_config<MODE_DENSE_MN>(block_n, ctas, pipes) && !find_config<MODE_DENSE_MN + 1>(block_n, ctas, pipes) &&
+      !find_config<MODE_DENSE_MN + 2>(block_n, ctas, pipes))
     return fail(DG_ERR_UNSUPPORTED, "block_n=%d with ctas=%d, pipes=%d is not built", block_n, ctas, pipes);
   t_force_bn = block_n;
   t_force_ctas = ctas;
@@ -673,14 +688,21 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
 
 int dg_get_device_error(void* stream, int* err) {
   if (!err) return fail(DG_ERR_NULL, "err must be non-NULL");
-  DG_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  // one reader at a time per process: the taken copy is a single word per device
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  auto st = static_cast<cudaStream_t>(stream);
+  // a plain launch (no programmatic serialisation): it starts after the stream's earlier kernels end
+  take_error_kernel<<<1, 1, 0, st>>>();
+  DG_CUDA_TRY(cudaGetLastError());
   int v = 0;
-  DG_CUDA_TRY(cudaMemcpyFromSymbol(&v, g_dg_error, sizeof(int)));
-  const int zero = 0;
-  DG_CUDA_TRY(cudaMemcpyToSymbol(g_dg_error, &zero, sizeof(int)));
+  DG_CUDA_TRY(cudaMemcpyFromSymbolAsync(&v, g_dg_error_taken, sizeof(int), 0, cudaMemcpyDeviceToHost, st));
+  DG_CUDA_TRY(cudaStreamSynchronize(st));
   *err = v;
   return DG_OK;
 }
+
+uint64_t dg_set_wait_limit_ns(uint64_t ns) { return g_wait_limit_ns.exchange(ns); }
 
 int dg_pack_sf_ue8m0(const float* sf, int32_t* packed, int batch, int mn, int kb, void* stream) {
   if (!sf || !packed) return fail(DG_ERR_NULL, "sf and packed must be non-NULL");

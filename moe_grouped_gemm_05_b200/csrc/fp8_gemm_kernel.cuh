@@ -88,7 +88,11 @@ constexpr int kThreadsFor = 32 * (8 + 3 * PIPES);
 constexpr int kThreads = kThreadsFor<1>;
 constexpr int kMaxMaskedGroups = 512;
 constexpr int kMaxSmem = 232448;                  // opt-in shared memory per block on sm_100
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+// Default limit of every pipeline wait: 2 s, far above any legitimate wait.
+// The main-loop waits take theirs from GemmArgs::wait_limit_ns (this value
+// unless the host changed it); the waits that drain copies and MMAs in
+// flight before a CTA exits always keep this one.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct GemmArgs {
   int rows;           // dense: M; contiguous: M_total; masked: M_max
@@ -109,6 +113,7 @@ struct GemmArgs {
   __nv_bfloat16* d;   // BF16 output (OUT_F32 == false)
   float* d32;         // FP32 output (OUT_F32 == true)
   const float* c;     // optional FP32 addend [rows][N] (OUT_F32 only), nullptr for none
+  uint64_t wait_limit_ns;  // limit of each main-loop wait before the CTA gives up
 };
 
 template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0, bool MASKED = true>
@@ -153,7 +158,7 @@ struct Layout {
   static constexpr int kOffEpi = ((kOffSft + PIPES * kSfRing * kSftBytes + 1023) / 1024) * 1024;
   static constexpr int kOffBar = kOffEpi + 8 * kEpiBuf;  // one staging buffer per epilogue warp
   static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 2 * PIPES * 4;
-  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag, 2 peer load counts
   static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
   static constexpr int kSmemBytes = kOffGroups + kGroupsBytes + 1024;
   static_assert(kSmemBytes <= kMaxSmem, "shared-memory budget exceeded");
@@ -196,7 +201,8 @@ __device__ __forceinline__ uint32_t pack_scale_word(const float* row, int kp, in
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting
 // (another role gave up) or this wait exceeded its limit (sets the error word).
 template <bool kCluster>
-__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                           uint64_t limit_ns) {
   auto probe = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (probe()) return true;
   const uint64_t t0 = global_timer_ns();
@@ -205,7 +211,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
     for (int i = 0; i < 32; ++i)
       if (probe()) return true;
     if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
+    if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(&g_dg_error, 0x10);
       return false;
@@ -307,6 +313,9 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
   uint64_t* sf_empty = sf_full + PIPES * L::kSfRing;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  // pairs: loads issued by the second CTA's producers, per pipeline (written into the first CTA)
+  uint32_t* peer_loads = reinterpret_cast<uint32_t*>(smem + L::kOffMisc + 8);
+  uint32_t prod_it = 0;  // loads issued by this warp's pipeline (producer warps)
   int* prefix = reinterpret_cast<int*>(smem + L::kOffGroups);
   int* counts = prefix + kMaxMaskedGroups + 1;
 
@@ -419,7 +428,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     // ============================================================ producer
     // Barrier of stage s in the MMA-issuing CTA, as a shared::cluster address.
     const uint32_t full0 = kPair ? mapa_shared(smem_u32(full_bar), 0) : smem_u32(full_bar);
-    uint32_t it = 0, li = 0;
+    uint32_t& it = prod_it;
+    uint32_t li = 0;
     bool ok = true;
     for (int t = unit0; t < ntiles && ok; t += units) {
       const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
@@ -438,7 +448,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const int kb_hi = min(num_kb, 4 * ge);
       for (int kb = 4 * gb; kb < kb_hi; ++kb, ++it) {
         const int s = sbase + static_cast<int>(it % L::kStagesPer);
-        ok = wait_phase<false>(&empty_bar[s], ((it / L::kStagesPer) & 1) ^ 1, abort_flag);
+        ok = wait_phase<false>(&empty_bar[s], ((it / L::kStagesPer) & 1) ^ 1, abort_flag, p.wait_limit_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         if (lane == 0) {
@@ -468,11 +478,20 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         }
       }
     }
-    // Drain: every load this CTA's barriers track must land before the CTA exits.
-    if (lane == 0 && (!kPair || rank == 0)) {
-      const uint32_t first = it > static_cast<uint32_t>(L::kStagesPer) ? it - L::kStagesPer : 0;
-      for (uint32_t i = first; i < it; ++i)
-        wait_phase_drain(&full_bar[sbase + i % L::kStagesPer], (i / L::kStagesPer) & 1);
+    // Drain: every load must land before its CTA exits.  One CTA waits for
+    // its last STAGES loads here (an earlier load's stage was consumed before
+    // a later load could reuse it).  In a pair every load signals the first
+    // CTA's barriers, and after an abort the two CTAs may have issued
+    // different counts: the second CTA publishes its count, and the first
+    // drains both after the cluster barrier of the teardown.
+    if constexpr (!kPair) {
+      if (lane == 0) {
+        const uint32_t first = it > static_cast<uint32_t>(L::kStagesPer) ? it - L::kStagesPer : 0;
+        for (uint32_t i = first; i < it; ++i)
+          wait_phase_drain(&full_bar[sbase + i % L::kStagesPer], (i / L::kStagesPer) & 1);
+      }
+    } else if (rank == 1 && lane == 0) {
+      st_shared_cluster_u32(mapa_shared(smem_u32(peer_loads + pipe), 0), it);
     }
     __syncwarp();
   } else if (is_issuer) {
@@ -519,7 +538,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         const uint32_t acc_use = (PIPES == 2 || L::kNumAcc == 1) ? own : (own >> 1);
         ++own;
         if (!mbar_try_wait(&tmem_empty[acc], (acc_use & 1) ^ 1))
-          ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag);
+          ok = wait_phase<false>(&tmem_empty[acc], (acc_use & 1) ^ 1, abort_flag, p.wait_limit_ns);
         if (!ok) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * L::kAccStride;
@@ -531,13 +550,13 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
           if (sf_group >= 2) {
             uint64_t* b = &sf_empty[rbase + (sf_group - 2) % L::kSfRing];
             const uint32_t par = ((sf_group - 2) / L::kSfRing) & 1;
-            if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag);
+            if (!mbar_try_wait(b, par)) ok = wait_phase<false>(b, par, abort_flag, p.wait_limit_ns);
           }
           // acquire at cluster scope: pairs with the scale producers' release (their
           // shared-memory writes are read by tcgen05.cp)
           if (ok && !(kPair ? mbar_try_wait_cluster(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1)
                             : mbar_try_wait(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1)))
-            ok = wait_phase<kPair>(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1, abort_flag);
+            ok = wait_phase<kPair>(&sf_full[rbase + ring], (sf_group / L::kSfRing) & 1, abort_flag, p.wait_limit_ns);
           if (!ok) break;
           tc_fence_after();
           {
@@ -553,7 +572,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
               if (!mbar_try_wait_addr(full_base + 8 * s, phase)) {
-                ok = wait_phase<false>(&full_bar[sbase + s], phase, abort_flag);
+                ok = wait_phase<false>(&full_bar[sbase + s], phase, abort_flag, p.wait_limit_ns);
                 if (!ok) break;
               }
               const uint64_t a_desc = (static_cast<uint64_t>(desc_hi) << 32) | (a_lo0 + s * (L::kABytes >> 4));
@@ -606,7 +625,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const int n0 = tl.n_blk * BN;
       for (int kp = gb; kp < ge; ++kp, ++group) {
         const uint32_t ring = group % L::kSfRing;
-        ok = wait_phase<false>(&sf_empty[rbase + ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag);
+        ok = wait_phase<false>(&sf_empty[rbase + ring], ((group / L::kSfRing) & 1) ^ 1, abort_flag, p.wait_limit_ns);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         // lane r gathers rows / columns r, r+32, r+64, r+96 of each 128-group
@@ -699,8 +718,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         acc_use = local_tile / L::kNumAcc;
       }
       ++local_tile;
-      bool ok = wait_phase<false>(&tmem_full[acc], acc_use & 1, abort_flag);
-      if (split && ok) ok = wait_phase<false>(&tmem_full[1], uses1++ & 1, abort_flag);
+      bool ok = wait_phase<false>(&tmem_full[acc], acc_use & 1, abort_flag, p.wait_limit_ns);
+      if (split && ok) ok = wait_phase<false>(&tmem_full[1], uses1++ & 1, abort_flag, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -850,7 +869,28 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
 
   // ---------------------------------------------------------------- teardown
   tc_fence_before();
-  if constexpr (kPair) cluster_sync(); else __syncthreads();
+  if constexpr (kPair) {
+    cluster_sync();  // both CTAs have stopped issuing; the second CTA's load counts are visible
+    if (rank == 0 && is_producer && lane == 0) {
+      // Phase j of a stage barrier completes with one arrival per CTA plus
+      // the bytes of both loads.  A CTA that gave up before issuing load j
+      // never arrives: arrive in its place, then wait for the loads that were
+      // issued.  Only the last STAGES phases can be incomplete.
+      const uint32_t it1 = *reinterpret_cast<volatile uint32_t*>(peer_loads + pipe);
+      const uint32_t hi = prod_it > it1 ? prod_it : it1;
+      const uint32_t lo = hi > static_cast<uint32_t>(L::kStagesPer) ? hi - L::kStagesPer : 0;
+      for (uint32_t j = lo; j < hi; ++j) {
+        uint64_t* b = &full_bar[sbase + j % L::kStagesPer];
+        if (j >= prod_it) mbar_arrive(b);
+        if (j >= it1) mbar_arrive(b);
+        wait_phase_drain(b, (j / L::kStagesPer) & 1);
+      }
+    }
+    __syncwarp();
+    cluster_sync();
+  } else {
+    __syncthreads();
+  }
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc<CTAS>(tmem_base, L::kTmemCols);

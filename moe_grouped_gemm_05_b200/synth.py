@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import dataclasses
 import math
+import os
 
 import numpy as np
 
@@ -53,12 +54,16 @@ def uniform01(seed: int, start: int, count: int) -> np.ndarray:
     return (z >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
 
 
-def normal(seed: int, count: int, sigma: float = 1.0, chunk: int = 1 << 24) -> np.ndarray:
-    """``count`` N(0, sigma) fp32 values (Box-Muller over consecutive pairs)."""
+def normal(seed: int, count: int, sigma: float = 1.0, chunk: int = 1 << 21) -> np.ndarray:
+    """``count`` N(0, sigma) fp32 values (Box-Muller over consecutive pairs).
+
+    Pair i uses stream outputs 2i and 2i+1 only, so chunks of pairs are drawn
+    independently (on a thread pool: NumPy's ufuncs release the GIL) and the
+    result does not depend on the chunking."""
     out = np.empty(count, dtype=np.float32)
     pairs = (count + 1) // 2
-    done = 0
-    while done < pairs:
+
+    def fill(done: int) -> None:
         n = min(chunk, pairs - done)
         u = uniform01(seed, 2 * done, 2 * n)
         u1 = 1.0 - u[0::2]  # (0, 1]
@@ -71,7 +76,16 @@ def normal(seed: int, count: int, sigma: float = 1.0, chunk: int = 1 << 24) -> n
         lo = 2 * done
         hi = min(count, lo + 2 * n)
         out[lo:hi] = z[: hi - lo].astype(np.float32)
-        done += n
+
+    starts = range(0, pairs, chunk)
+    if pairs <= chunk:
+        for s in starts:
+            fill(s)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
     return out
 
 

@@ -9,6 +9,9 @@ Integer-valued problems must match bit for bit.
 """
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -78,3 +81,20 @@ def check_close(got_bits: np.ndarray, ref_bits: np.ndarray, what: str = ""):
     den = float((x * x + y * y).sum())
     diff = 0.0 if den == 0 else 1.0 - 2.0 * float((x * y).sum()) / den
     assert diff < 1e-4, f"{what}: normalised difference {diff}"
+
+
+def oracle_rows(a, sfa_words, b, sfb_words, M, N, K, rows, chunk: int = 256) -> np.ndarray:
+    """The oracle's BF16 bits of the given output rows of D = A . B^T, computed
+    in chunks of rows on a thread pool with single-threaded BLAS (each chunk
+    is an independent call of the oracle, so the result is the same as one
+    call over all rows)."""
+    from threadpoolctl import threadpool_limits
+
+    rows = np.asarray(rows)
+    if len(rows) <= chunk:
+        return oracle.fp8_gemm_nt(a, sfa_words, b, sfb_words, M, N, K, rows=rows)
+    parts = [rows[i:i + chunk] for i in range(0, len(rows), chunk)]
+    with threadpool_limits(1):
+        with ThreadPoolExecutor(max_workers=max(1, min(32, os.cpu_count() or 1))) as ex:
+            out = list(ex.map(lambda r: oracle.fp8_gemm_nt(a, sfa_words, b, sfb_words, M, N, K, rows=r), parts))
+    return np.concatenate(out)

@@ -86,6 +86,31 @@ def test_config_override(lib):
     assert lib.dg_set_config(0, 0, 0) == 0
 
 
+def test_wait_limit_knob(lib):
+    """The pipeline-wait limit is process-wide host state: the setter returns
+    the previous value, and the default is 2 s."""
+    prev = binding.set_wait_limit_ns(0)
+    assert prev == 2_000_000_000
+    assert binding.set_wait_limit_ns(123) == 0
+    assert binding.set_wait_limit_ns(prev) == 123
+    with pytest.raises(ValueError):
+        binding.set_wait_limit_ns(-1)
+
+
+def test_forced_tile_falls_back_per_entry_point(lib):
+    """A forced tile that one entry point does not build leaves that entry
+    point on the heuristic instead of failing its calls."""
+    from moe_grouped_gemm_05_b200 import binding as dg
+
+    heur = dg.describe_config("contiguous", 32768, 4096, 7168, 8)
+    assert lib.dg_set_config(64, 1, 1) == 0      # built for dense / masked only
+    try:
+        assert dg.describe_config("contiguous", 32768, 4096, 7168, 8) == heur
+        assert dg.describe_config("dense", 4096, 7168, 2048).startswith("128x64x")
+    finally:
+        assert lib.dg_set_config(0, 0, 0) == 0
+
+
 def test_heuristic_choices_without_gpu(lib):
     """The configuration heuristic is host logic: without a device it assumes
     148 SMs.  Decode-sized dense problems take split-K tiles over two

@@ -70,3 +70,36 @@ def test_committed_traffic_records_are_consistent():
     for e in rec.values():
         assert e["dram_bytes_per_launch"] == e["dram_read_bytes"] + e["dram_write_bytes"]
         assert e["kernel_hash"] and e["kernel_config"] and os.path.exists(os.path.join(ROOT, e["source"].split()[0]))
+
+
+def _contig_problem():
+    from moe_grouped_gemm_05_b200 import synth
+
+    return synth.contiguous_problem(5, 384, 256, rows=700, seed=11)
+
+
+def test_shard_problem_n_split_covers_every_column_once():
+    from moe_grouped_gemm_05_b200 import synth
+
+    p = synth.dense_problem(64, 1408, 256, seed=3)
+    parts = [bench.shard_problem(p, 3, r, "n") for r in range(3)]
+    assert sum(q.N for q in parts) == p.N and all(q.N % 128 == 0 for q in parts)
+    assert np.array_equal(np.concatenate([q.b for q in parts]), p.b)
+    assert np.array_equal(np.concatenate([q.sfb for q in parts]), p.sfb)
+    assert sum(q.flops for q in parts) == p.flops
+    assert bench.shard_problem(p, 1, 0, "n") is p
+
+
+def test_shard_problem_experts_keeps_every_valid_row_once():
+    p = _contig_problem()
+    seen = []
+    for r in range(2):
+        q = bench.shard_problem(p, 2, r, "experts")
+        assert q.M % 128 == 0 and q.a.shape == (q.M, p.K) and q.b.shape[0] == q.G
+        valid = q.m_indices >= 0
+        # every local row holds one of the global rows of an owned expert, with its codes and scales
+        for i in np.nonzero(valid)[0][:50]:
+            j = np.nonzero((p.a == q.a[i]).all(axis=1))[0]
+            assert len(j) >= 1 and p.m_indices[j[0]] >= 0
+        seen.append(int(valid.sum()))
+    assert sum(seen) == p.valid_rows

@@ -1,10 +1,10 @@
 """Parity at the benchmark workloads' full sizes, in the launch configuration
 the benchmark uses (the heuristic's choice, scales packed on the GPU).
 
-The oracle recomputes sampled output rows (first/last rows, tile and expert
-boundaries, outlier rows, random rows) in full; properties that hold at any
-size (finite outputs, untouched padding / masked rows, bit-exact scale
-packing) are checked over the whole output.
+Every valid output row of all five workloads is recomputed by the oracle
+(on a thread pool, a chunk of rows per call) and compared element by element
+within the BF16 tolerance; padding rows of the contiguous layout and masked
+rows keep their sentinel bit pattern, and the scale packing is bit-exact.
 """
 import numpy as np
 import pytest
@@ -14,7 +14,7 @@ import oracle
 from moe_grouped_gemm_05_b200 import binding as dg
 from moe_grouped_gemm_05_b200 import synth
 
-from helpers import bits, check_close
+from helpers import bits, check_close, oracle_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -41,14 +41,12 @@ def _pack_on_gpu(sf: np.ndarray):
     return got if sf.ndim == 3 else got[0], (ref if sf.ndim == 3 else ref[0])
 
 
-def _sample_rows(M, rng, extra=()):
-    base = {0, 1, 127, 128, 255, 256, M // 2, M - 129, M - 128, M - 2, M - 1, *extra}
-    base |= set(rng.integers(0, M, size=12).tolist())
-    return np.array(sorted(r for r in base if 0 <= r < M))
-
-
 def _fp8(x):
     return torch.from_numpy(x).cuda().view(torch.float8_e4m3fn)
+
+
+def _sentinel(shape):
+    return torch.from_numpy(np.full(shape, SENTINEL, np.uint16).view(np.int16)).cuda().view(torch.bfloat16)
 
 
 @pytest.mark.parametrize("name", ["dense_4096x7168x2048", "dense_64x7168x2048", "dense_8192x8192x8192_outliers"])
@@ -60,55 +58,52 @@ def test_dense_full_size(name):
     torch.cuda.synchronize()
     assert dg.get_device_error() == 0
     got = bits(d)
-    assert np.isfinite(oracle.bf16_bits_to_f64(got)).all()
-    rng = np.random.default_rng(7)
-    extra = ()
+    ref = oracle_rows(p.a, sa, p.b, sb, p.M, p.N, p.K, np.arange(p.M))
+    check_close(got, ref, name)
     if "outliers" in name:
-        # rows scaled by 64 before quantisation (the same draw as the generator's)
-        extra = tuple(synth.choose_rows(1004 ^ 0x5A5A, p.M, int(round(0.01 * p.M)))[:6].tolist())
-    rows = np.arange(p.M) if p.M <= 64 else _sample_rows(p.M, rng, extra)
-    ref = oracle.fp8_gemm_nt(p.a, sa, p.b, sb, p.M, p.N, p.K, rows=rows)
-    check_close(got[rows], ref, name)
+        # the rows scaled by 64 before quantisation (the generator's own draw) are among them
+        out = synth.choose_rows(1004 ^ 0x5A5A, p.M, int(round(0.01 * p.M)))
+        assert len(out) == 82
+        check_close(got[out], ref[out], f"{name}: outlier rows")
 
 
 def test_contiguous_full_size():
     p = synth.WORKLOADS["contiguous_8x4096x7168_zipf1.1"]()
     sfa, sa = _pack_on_gpu(p.sfa)
     sfb, sb = _pack_on_gpu(p.sfb)
-    d = torch.from_numpy(np.full((p.M, p.N), SENTINEL, np.uint16).view(np.int16)).cuda().view(torch.bfloat16)
+    d = _sentinel((p.M, p.N))
     dg.m_grouped_fp8_gemm_nt_contiguous(_fp8(p.a), sfa, _fp8(p.b), sfb, torch.from_numpy(p.m_indices).cuda(), d)
     torch.cuda.synchronize()
     assert dg.get_device_error() == 0
     got = bits(d)
     pad = p.m_indices < 0
     assert (got[pad] == SENTINEL).all(), "padding rows were written"
-    assert np.isfinite(oracle.bf16_bits_to_f64(got[~pad])).all()
-    rng = np.random.default_rng(8)
-    rows = []
+    ref = np.full_like(got, SENTINEL)
     for e in range(p.G):
-        idx = np.nonzero(p.m_indices == e)[0]
-        rows += [idx[0], idx[-1], *rng.choice(idx, size=3, replace=False)]
-    rows = np.array(sorted(set(int(r) for r in rows)))
-    for e in range(p.G):
-        re = rows[p.m_indices[rows] == e]
-        ref = oracle.fp8_gemm_nt(p.a, sa, p.b[e], sb[e], p.M, p.N, p.K, rows=re)
-        check_close(got[re], ref, f"contiguous expert {e}")
+        rows = np.nonzero(p.m_indices == e)[0]
+        assert len(rows) > 0
+        ref[rows] = oracle_rows(p.a, sa, p.b[e], sb[e], p.M, p.N, p.K, rows)
+        check_close(got[rows], ref[rows], f"contiguous expert {e}")
+    # the whole call's normalised difference, over every valid row
+    check_close(got[~pad], ref[~pad], "contiguous, all valid rows")
 
 
 def test_masked_full_size():
     p = synth.WORKLOADS["masked_16x256x7168x2048"]()
     sfa, sa = _pack_on_gpu(p.sfa)
     sfb, sb = _pack_on_gpu(p.sfb)
-    d = torch.from_numpy(np.full((p.G, p.M, p.N), SENTINEL, np.uint16).view(np.int16)).cuda().view(torch.bfloat16)
+    d = _sentinel((p.G, p.M, p.N))
     dg.m_grouped_fp8_gemm_nt_masked(_fp8(p.a), sfa, _fp8(p.b), sfb, torch.from_numpy(p.masked_m).cuda(), d)
     torch.cuda.synchronize()
     assert dg.get_device_error() == 0
     got = bits(d)
-    rng = np.random.default_rng(9)
+    valid_got, valid_ref = [], []
     for g, mg in enumerate(p.masked_m):
         assert (got[g, mg:] == SENTINEL).all(), f"expert {g}: masked rows were written"
         if mg == 0:
             continue
-        rows = np.array(sorted({0, mg - 1, *rng.integers(0, mg, size=2).tolist()}))
-        ref = oracle.fp8_gemm_nt(p.a[g], sa[g], p.b[g], sb[g], p.M, p.N, p.K, rows=rows)
-        check_close(got[g, rows], ref, f"masked expert {g}")
+        ref = oracle_rows(p.a[g], sa[g], p.b[g], sb[g], p.M, p.N, p.K, np.arange(mg))
+        check_close(got[g, :mg], ref, f"masked expert {g}")
+        valid_got.append(got[g, :mg])
+        valid_ref.append(ref)
+    check_close(np.concatenate(valid_got), np.concatenate(valid_ref), "masked, all valid rows")
