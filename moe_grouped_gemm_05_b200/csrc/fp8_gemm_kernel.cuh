@@ -200,16 +200,17 @@ __device__ __forceinline__ uint32_t pack_scale_word(const float* row, int kp, in
 
 // Bounded wait on an mbarrier phase.  Returns false when the CTA is aborting
 // (another role gave up) or this wait exceeded its limit (sets the error word).
+// A plain try_wait may keep the thread suspended until the phase completes,
+// so every probe here carries a suspend-time hint (kPollNs): the loop looks
+// at the clock and the abort flag at least that often.
+constexpr uint32_t kPollNs = 1000;
 template <bool kCluster>
 __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                            uint64_t limit_ns) {
-  auto probe = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
-  if (probe()) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (probe()) return true;
+    if (kCluster ? mbar_try_wait_cluster_hint(bar, parity, kPollNs) : mbar_try_wait_hint(bar, parity, kPollNs))
+      return true;
     if (*abort_flag) return false;
     if (global_timer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
@@ -222,7 +223,7 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, volat
 // Wait used while draining at exit: ignores the abort flag, still bounded.
 __device__ __forceinline__ void wait_phase_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_hint(bar, parity, kPollNs)) {
     if (global_timer_ns() - t0 > kWaitLimitNs) {
       atomicOr(&g_dg_error, 0x10);
       return;
