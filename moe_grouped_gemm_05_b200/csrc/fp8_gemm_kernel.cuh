@@ -276,6 +276,21 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
   return tl;
 }
 
+// N width of the MMAs of a tile.  A ragged last N tile (fewer than BN columns
+// of D left) runs narrower MMAs, so the tensor core does not compute columns
+// that are never stored.  Only widths that built configurations use already
+// are taken: 64 (one CTA) and 128.  An MN-major B tile keeps its width (its
+// loads are whole 128-column boxes).
+template <int BN, int CTAS, int LAYOUT>
+__device__ __forceinline__ int tile_mma_n(int n0, int N) {
+  if constexpr ((LAYOUT & 2) != 0) return BN;
+  const int rem = N - n0;
+  if (rem >= BN) return BN;
+  if (CTAS == 1 && BN > 64 && rem <= 64) return 64;
+  if (BN > 128 && rem <= 128) return 128;
+  return BN;
+}
+
 // Expert of a contiguous-layout tile, or -1 when the tile has nothing to
 // compute: its (first) block starts with a padding row or an out-of-range
 // index, or it is a second-pass pair whose blocks share one expert.
@@ -455,7 +470,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         if (lane == 0) {
           uint8_t* a_dst = smem + L::kOffA + s * L::kABytes;
           uint8_t* b_dst = smem + L::kOffB + s * L::kBBytes;
-          const int b_row = n0 + static_cast<int>(rank) * L::kBRows;
+          // each CTA of a pair holds half of the tile's MMA width of B
+          const int b_row = n0 + static_cast<int>(rank) * (tile_mma_n<BN, CTAS, LAYOUT>(n0, p.N) / CTAS);
           // K-major boxes are (K, rows); MN-major boxes are (rows, K), 128 x 128 each
           const int ax = kAmn ? m_base : kb * kBK, ay = kAmn ? kb * kBK : m_base;
           if constexpr (kPair) tma_load_3d_pair(a_dst, &tm_a, full0 + 8 * s, ax, ay, grp_a);
@@ -512,7 +528,6 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const uint32_t b_lo0 = static_cast<uint32_t>(
           make_smem_desc(smem_u32(smem + L::kOffB + sbase * L::kBBytes), kBmn ? 128 * kBK : 16, 1024, 2));
       const uint32_t desc_hi = static_cast<uint32_t>(make_smem_desc(0, 16, 1024, 2) >> 32);
-      const uint32_t idesc0 = make_idesc_mxf8(L::kTileM, BN, 0, 0, kAmn, kBmn);
       // start-address step per K = 32 (address field in 16-byte units): K-major,
       // +32 B inside the swizzled 128-byte row; MN-major, +4 atoms of 8 K-rows
       constexpr uint32_t kAStep = kAmn ? 256 : 2, kBStep = kBmn ? 256 : 2;
@@ -527,12 +542,13 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const uint32_t sft_hi = static_cast<uint32_t>(make_smem_desc(0, 128, 256, 0) >> 32);
       const uint32_t sfx_hi = static_cast<uint32_t>(make_smem_desc(0, 0, 128, 0) >> 32);
       for (int t = unit0; t < ntiles && ok; t += units) {
-        if (MODE == MODE_CONTIG) {  // only the contiguous layout can skip a tile
-          const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
-          if (contig_expert<CTAS>(tl, p) < 0) continue;
-        }
+        const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
+        // only the contiguous layout can skip a tile
+        if (MODE == MODE_CONTIG && contig_expert<CTAS>(tl, p) < 0) continue;
         int gb, ge;
         if (!plan(li, gb, ge)) continue;
+        const uint32_t idesc_t =
+            make_idesc_mxf8(L::kTileM, tile_mma_n<BN, CTAS, LAYOUT>(tl.n_blk * BN, p.N), 0, 0, kAmn, kBmn);
         const int kb_hi = min(num_kb, 4 * ge);
         // one pipeline: alternate accumulators; two: accumulator = pipeline
         const uint32_t acc = PIPES == 2 ? pipe : (L::kNumAcc == 1 ? 0 : (own & 1));
@@ -568,7 +584,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
                                                            (lo + (L::kSftMainBytes >> 4)));
           }
           const int nk = min(4, kb_hi - kb0);
-          uint32_t id = idesc0;
+          uint32_t id = idesc_t;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
