@@ -290,23 +290,90 @@ static const Config* find_config(int bn, int ctas, int pipes = 0) {
 static thread_local int t_force_ctas = 0;
 static thread_local int t_force_pipes = 0;
 
-// Heuristic.  Each configuration has a sustained rate measured on B200 with
-// full waves and cold L2 (dense 4096x7168x2048, 8192^3, contiguous and
-// masked workloads, FP8 TFLOP/s).  Every tcgen05 instruction costs the
-// thread that issues it a fixed ~60-70 cycles, so one issuing thread keeps
-// the tensor pipe only ~65% busy on 224-wide tiles and less on 128-wide
-// ones.  Two pipelines per CTA (two issuing threads, alternate tiles)
-// remove that bound; they pay off with 2-CTA tiles, which also halve the B
-// bytes each SM loads from L2.  The estimated time of a configuration is
-// its padded work (whole tiles, whole waves of co-resident units) divided by
-// that rate.  Problems of at most 128 rows stream B from HBM and run fastest
-// on the configuration with the most CTAs, so they keep 1-CTA tiles; so
-// does the masked layout, where a 256-row tile wastes half its work on
-// experts with <= 128 rows.
-static double config_rate(const Config& c) {
-  if (c.bn <= 128) return c.ctas == 2 ? (c.pipes == 2 ? 2000.0 : 1400.0) : 1550.0;
-  if (c.bn <= 224) return c.ctas == 2 ? (c.pipes == 2 ? 2700.0 : 2300.0) : 2400.0;
-  return c.ctas == 2 ? 2100.0 : 2250.0;
+// Heuristic: a cost model fitted to measurements on B200.  A configuration
+// spends, per tile of a CTA (or CTA pair), kb_ns per 128-wide K block plus
+// tile_ns for the rest (first loads, epilogue drain, tile switch); a problem
+// costs (tiles / units) such tiles, at least one, so both the K depth and the
+// N tile count enter.  Problems that stream more bytes than that time can
+// carry are bound by HBM instead: max(compute, bytes / kHbmBytesPerNs).
+// The constants were fitted to CUDA-event timings of every built
+// configuration, back to back under the 1 kW power cap, on dense
+// 4096x7168x2048 (K = 2048) and 8192^3 (K = 8192), and checked against the
+// contiguous 8 x (4096 x 7168) workload (within 3 %) and the masked and
+// 64-row decode workloads (the model's pick is the fastest measured).
+// Every tcgen05 instruction costs the thread that issues it ~60 cycles, so
+// narrow tiles pay more per FLOP (kb_ns of a 128-wide tile is not half that
+// of a 256-wide one); 2-CTA tiles halve the B bytes an SM loads; two
+// pipelines per CTA hide one issuing thread's overhead behind the other's.
+struct CostParams {
+  int bn, ctas, pipes;
+  bool splitk;
+  double kb_ns, tile_ns;
+};
+// The contiguous layout's tiles run slower per K block than dense ones when
+// the experts' weights exceed L2 (8 x 4096 x 7168 bytes here), most of all
+// the 1-CTA 224-wide tile, which loads twice the B bytes of a 2-CTA tile per
+// SM; its kb_ns are fitted on that workload (interleaved runs), tile_ns kept.
+// The 256-wide tile has one accumulator, which its epilogue releases as soon
+// as it has been read: its tile_ns is that of the interleaved runs.
+static const CostParams kCostContig[] = {
+    {128, 1, 1, false, 363, 757}, {224, 1, 1, false, 531, 1345}, {256, 1, 1, false, 517, 2250},
+    {224, 2, 2, false, 434, 2023},
+};
+static const CostParams kCost[] = {
+    {128, 1, 1, false, 360, 757},  {224, 1, 1, false, 453, 1345}, {256, 1, 1, false, 514, 2566},
+    {128, 2, 1, false, 366, 1095}, {224, 2, 1, false, 442, 1865}, {256, 2, 1, false, 482, 3280},
+    {224, 2, 2, false, 408, 2023}, {128, 2, 2, false, 286, 1186}, {64, 1, 1, false, 313, 577},
+    {64, 1, 2, true, 387, 959},    {128, 1, 2, true, 680, 1288},
+};
+// Sustained HBM read+write rate of a streaming GEMM (the masked workload's measured 5.4 TB/s), bytes per ns.
+constexpr double kHbmBytesPerNs = 5400.0;
+
+template <int MODE>
+static const CostParams* cost_params(const Config& c) {
+  if (MODE == MODE_CONTIG)
+    for (const CostParams& k : kCostContig)
+      if (k.bn == c.bn && k.ctas == c.ctas && k.pipes == c.pipes && k.splitk == c.splitk) return &k;
+  const CostParams* best = nullptr;
+  for (const CostParams& k : kCost) {
+    if (k.bn == c.bn && k.ctas == c.ctas && k.pipes == c.pipes && k.splitk == c.splitk) return &k;
+    if (k.bn == c.bn && k.ctas == c.ctas && !best) best = &k;  // layouts / FP32 output: same tile shape
+  }
+  return best;
+}
+
+// Estimated time (ns) of configuration c.  rows_est: rows of the problem
+// (masked: the expected valid rows); groups: experts (contiguous, masked).
+template <int MODE>
+static double config_cost(const Config& c, long long rows_est, int N, int K, int sms, int groups) {
+  const CostParams* k = cost_params<MODE>(c);
+  if (!k) return 1e300;
+  const long long tile_m = 128LL * c.ctas;
+  long long m_tiles;
+  if (MODE == MODE_MASKED) {
+    const long long per = std::max<long long>(1, rows_est / std::max(1, groups));
+    m_tiles = static_cast<long long>(groups) * ((per + tile_m - 1) / tile_m);
+  } else {
+    m_tiles = (rows_est + tile_m - 1) / tile_m;
+    if (MODE == MODE_CONTIG && c.ctas == 2) m_tiles += groups;  // second-pass pairs at expert boundaries
+  }
+  // the last N tile runs a narrower MMA when it is ragged (64 or 128 columns)
+  const int full = N / c.bn, rem = N - full * c.bn;
+  double n_tiles = full;
+  if (rem > 0) {
+    const int nt = (c.ctas == 1 && c.bn > 64 && rem <= 64) ? 64 : ((c.bn > 128 && rem <= 128) ? 128 : c.bn);
+    n_tiles += static_cast<double>(nt) / c.bn;
+  }
+  const double units = std::max(1, sms / c.ctas);
+  const double waves = std::max(1.0, static_cast<double>(m_tiles) * n_tiles / units);
+  const double kb = (K / 128) * (c.splitk ? 0.5 : 1.0);
+  const double compute = waves * (kb * k->kb_ns + k->tile_ns);
+  const double experts = MODE == MODE_DENSE ? 1.0 : groups;
+  const double bytes = static_cast<double>(rows_est) * (K + 2.0 * N) + experts * static_cast<double>(N) * K;
+  const double memory = bytes / kHbmBytesPerNs;
+  // the smaller term is not fully hidden behind the larger one (first loads,
+  // last epilogue): a tenth of it breaks ties between HBM-bound configurations
+  return std::max(compute, memory) + 0.1 * std::min(compute, memory);
 }
 
 template <int MODE>
@@ -316,27 +383,16 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms, in
   if (t_force_bn) {
     if (const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes)) return f;
   }
-  (void)K;
   int n = 0;
   const Config* t = config_table<MODE>(&n);
   const Config* best = nullptr;
   double best_cost = 1e300;
   for (int i = 0; i < n; ++i) {
     const Config& c = t[i];
-    if ((MODE == MODE_MASKED || MODE == MODE_DENSE_F32 || rows_est <= 128) && c.ctas != 1) continue;
-    // split-K tiles keep no second accumulator for overlap: only for a single M block
-    // (decode), and only when K has at least two groups of 4 K blocks
-    if (c.splitk && (rows_est > 128 || K <= 4 * 128)) continue;
-    const long long tile_m = 128LL * c.ctas;
-    long long m_tiles = (rows_est + tile_m - 1) / tile_m;
-    if (MODE == MODE_CONTIG && c.ctas == 2) m_tiles += groups;  // second-pass pairs at expert boundaries
-    const long long n_tiles = (N + c.bn - 1) / c.bn;
-    const long long units = std::max(1, sms / c.ctas);
-    const long long tiles = m_tiles * n_tiles;
-    const long long waves = (tiles + units - 1) / units;
-    // padded work in units of 128x128 tile-K-blocks, spread over the whole grid
-    const double work = static_cast<double>(waves) * units * (tile_m / 128.0) * (c.bn / 128.0);
-    const double cost = work / config_rate(c) * (c.splitk ? 0.5 : 1.0);  // split-K halves the K loop
+    // split-K tiles keep no second accumulator for overlap; they need at least two groups of 4 K blocks
+    if (c.splitk && K <= 4 * 128) continue;
+    const double cost = config_cost<MODE == MODE_CONTIG || MODE == MODE_MASKED ? MODE : MODE_DENSE>(
+        c, rows_est, N, K, sms, groups);
     if (cost < best_cost * 0.999) {
       best_cost = cost;
       best = &c;
@@ -674,7 +730,7 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
   long long tiles = 0;
   if (kind == 2) {
     const long long est = std::max<long long>(1, static_cast<long long>(num_groups) * M / 2);
-    c = choose_config<MODE_MASKED>(est, N, K, sms);
+    c = choose_config<MODE_MASKED>(est, N, K, sms, num_groups);
     if (c) tiles = static_cast<long long>(num_groups) * ((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   } else {
     c = kind == 1 ? choose_config<MODE_CONTIG>(M, N, K, sms, num_groups) : choose_config<MODE_DENSE>(M, N, K, sms);
@@ -925,7 +981,7 @@ static int masked_impl(const void* a, const void* sfa, const void* b, const int3
   if ((r = device_info(&di))) return r;
   // the device decides the real tile count; the heuristic assumes half-full experts
   const long long rows_est = std::max<long long>(1, static_cast<long long>(num_groups) * M_max / 2);
-  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, usable_sms(di.sms));
+  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, usable_sms(di.sms), num_groups);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
   if ((r = build_maps_cached(maps, cfg, a, b, d, M_max, num_groups, N, K, num_groups, M_max, num_groups)))

@@ -541,14 +541,20 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const uint32_t sf_slot0 = tmem_base + L::kSfBaseCol + pipe * 2 * L::kSfSlotCols;
       const uint32_t sft_hi = static_cast<uint32_t>(make_smem_desc(0, 128, 256, 0) >> 32);
       const uint32_t sfx_hi = static_cast<uint32_t>(make_smem_desc(0, 0, 128, 0) >> 32);
+      const uint32_t idesc_full = make_idesc_mxf8(L::kTileM, BN, 0, 0, kAmn, kBmn);
+      const bool ragged_n = p.N % BN != 0;
       for (int t = unit0; t < ntiles && ok; t += units) {
-        const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
-        // only the contiguous layout can skip a tile
-        if (MODE == MODE_CONTIG && contig_expert<CTAS>(tl, p) < 0) continue;
+        // the tile itself is needed only to skip contiguous tiles and to narrow a ragged last N tile
+        int n0 = 0;
+        if (MODE == MODE_CONTIG || ragged_n) {
+          const Tile tl = tile_of<MODE, L::kTileM>(t, p, prefix, counts);
+          if (MODE == MODE_CONTIG && contig_expert<CTAS>(tl, p) < 0) continue;
+          n0 = tl.n_blk * BN;
+        }
         int gb, ge;
         if (!plan(li, gb, ge)) continue;
         const uint32_t idesc_t =
-            make_idesc_mxf8(L::kTileM, tile_mma_n<BN, CTAS, LAYOUT>(tl.n_blk * BN, p.N), 0, 0, kAmn, kBmn);
+            ragged_n ? make_idesc_mxf8(L::kTileM, tile_mma_n<BN, CTAS, LAYOUT>(n0, p.N), 0, 0, kAmn, kBmn) : idesc_full;
         const int kb_hi = min(num_kb, 4 * ge);
         // one pipeline: alternate accumulators; two: accumulator = pipeline
         const uint32_t acc = PIPES == 2 ? pipe : (L::kNumAcc == 1 ? 0 : (own & 1));
@@ -708,6 +714,8 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     const uint32_t empty0 = kPair ? mapa_shared(smem_u32(tmem_empty), 0) : smem_u32(tmem_empty);
     constexpr int kChunks = BN / 32;
     constexpr int kMaxMine = (kChunks + 1) / 2;
+    // a single accumulator (no split tiles: one pipeline) with BF16 output releases it early
+    constexpr bool kEarlyRelease = !OUT_F32 && L::kNumAcc == 1 && PIPES == 1;
     const int nmine = half == 0 ? (kChunks + 1) / 2 : kChunks / 2;
     uint32_t local_tile = 0;
     uint32_t uses0 = 0, uses1 = 0;  // tiles that used accumulator 0 / 1 so far (two pipelines)
@@ -842,6 +850,67 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         }
       };
 
+      if constexpr (kEarlyRelease) {
+        // One accumulator: the next tile's MMAs wait for it, so it is handed
+        // back as soon as it has been read.  The warp's chunks go from TMEM
+        // to packed BF16 in registers, the accumulator is released, and only
+        // then are they staged and stored.
+        uint32_t pk[kMaxMine][16];
+        if (any_valid) {
+#pragma unroll
+          for (int i = 0; i < kMaxMine; ++i) {
+            const int c = half + 2 * i;
+            if (i < nmine && n0 + 32 * c < p.N) {
+              uint32_t r[32];
+              tmem_ld_32x32b_x32(t_row + 32 * c, r);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * j]), __uint_as_float(r[2 * j + 1]));
+                pk[i][j] = *reinterpret_cast<uint32_t*>(&h2);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_remote(empty0 + 8 * acc);
+          else mbar_arrive(&tmem_empty[acc]);
+        }
+        if (any_valid) {
+#pragma unroll
+          for (int i = 0; i < kMaxMine; ++i) {
+            const int col0 = n0 + 32 * (half + 2 * i);
+            if (i >= nmine || col0 >= p.N) break;
+            if (all_valid) {
+              if (lane == 0) bulk_wait_group_read<0>();  // previous store has read the buffer
+              __syncwarp();
+              uint8_t* rowp = buf + lane * 64;
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const int chunk = v ^ ((lane >> 1) & 3);  // 64-byte swizzle
+                *reinterpret_cast<uint4*>(rowp + chunk * 16) =
+                    make_uint4(pk[i][4 * v], pk[i][4 * v + 1], pk[i][4 * v + 2], pk[i][4 * v + 3]);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tm_d, buf, col0, row0, zd);
+                bulk_commit_group();
+              }
+            } else if (valid) {
+              __nv_bfloat16* dst = p.d + row_g * p.N + col0;
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                if (col0 + 8 * v < p.N)
+                  *reinterpret_cast<uint4*>(dst + 8 * v) =
+                      make_uint4(pk[i][4 * v], pk[i][4 * v + 1], pk[i][4 * v + 2], pk[i][4 * v + 3]);
+            }
+          }
+        }
+        continue;
+      }
       if (any_valid) {
         uint32_t r[2][32];
         if (nmine > 0 && n0 + 32 * half < p.N) tmem_ld_32x32b_x32(t_row + 32 * half, r[0]);
@@ -880,7 +949,9 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         }
       }
     }
-    if (lane == 0) bulk_wait_group<0>();
+    // Before the CTA exits its staging buffers must have been read out; the
+    // global writes themselves complete with the grid.
+    if (lane == 0) bulk_wait_group_read<0>();
     __syncwarp();
   }
 

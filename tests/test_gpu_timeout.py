@@ -35,7 +35,9 @@ def _gpu():
 
 @pytest.mark.parametrize("cfg", [(128, 1, 1), (64, 1, 2)])
 def test_wait_that_runs_out_reports_timeout_and_next_call_is_correct(cfg):
-    M, N, K = 128, 512, 2048  # 16 K blocks: split-K applies to the (64, 1, 2) tile
+    # 256 K blocks: the epilogue's first wait (a whole tile's K loop, tens of
+    # microseconds) outlasts any suspended probe and the clock's granularity
+    M, N, K = 128, 512, 32768
     p = synth.dense_problem(M, N, K, seed=4242)
     sa, sb = packed(p)
     t = to_device(p, sa, sb)
