@@ -642,7 +642,10 @@ def run_ours(args):
                    "l2": (f"inputs rotate over {m['nsets']} device copies "
                           f"({m['nsets'] * m['per_set'] / 1e6:.0f} MB > 2x L2)")},
         "roofline": roof,
+        # this library's launches in one replay of the K steps (the replay whose time is ms_per_step x steps)
         "gpu_launches": (1 if args.fused_pack else 2) * args.steps,
+        "gpu_launches_note": (f"per replay of the {args.steps} steps; the reported time is the median of "
+                              f"{m['replays']} replays"),
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "device_error": m["device_error"],
     }
