@@ -68,6 +68,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end loop (0 = min(steps, 100))")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end loop (profiling runs)")
     ap.add_argument("--eager", action="store_true", help="time host-issued launches instead of a CUDA graph")
+    ap.add_argument("--no-library", action="store_true", help="skip the cuBLAS context timing of dense workloads")
     ap.add_argument("--fused-pack", action="store_true",
                     help="let the GEMM read A's fp32 scales and pack them itself instead of a packing launch")
     return ap.parse_args()
@@ -464,11 +465,50 @@ def measure(p, dg, lib, torch, args, dev, local, barrier):
     gemm_ms, gemm_reps = timed("gemm", gemm_only)
     sampler.stop()
     err = dg.get_device_error()
+    library = library_context(p, sets, torch, args, timed, graphs) if p.kind == "dense" else None
     m = Measured(p=p, sets=sets, per_set=per_set, nsets=nsets, kernel_desc=kernel_desc,
                  step_ms=step_ms / K, gemm_ms=gemm_ms / K, replays=step_reps, gemm_replays=gemm_reps,
-                 window_ms=step_ms * step_reps, clocks=sampler.summary(), device_error=err)
+                 window_ms=step_ms * step_reps, clocks=sampler.summary(), device_error=err, library=library)
     del graphs
     return m
+
+
+def library_context(p, sets, torch, args, timed, graphs):
+    """cuBLAS's FP8 GEMM on the same operands, timed the same way, for context.
+
+    PyTorch's _scaled_mm reaches cuBLAS's 1x128 / 128x128 block-scaled FP8
+    GEMM only when built against CUDA 12.9 or later; otherwise the closest
+    library GEMM is the per-tensor-scaled FP8 one (one scale per operand: less
+    work than the block-scaled recipe, so a generous reference).  Never part
+    of the measured path; null with the reason when unavailable."""
+    if args.eager or args.no_library:
+        return None
+    try:
+        K = args.steps
+        one = torch.ones((), device="cuda")
+        ops = [(s["a"], s["b"]) for s in sets]
+
+        def call(i):
+            a, b = ops[i % len(ops)]
+            torch._scaled_mm(a, b.t(), one, one, out_dtype=torch.bfloat16)
+
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(cap):
+            for i in range(3):
+                call(i)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                for i in range(K):
+                    call(i)
+        torch.cuda.synchronize()
+        graphs["library"] = g
+        ms, reps = timed("library", None)
+        return {"library": "cuBLAS FP8 GEMM through torch._scaled_mm, per-tensor scales (the block-scaled "
+                           "recipe needs CUDA 12.9 in PyTorch's build)", "kernel_ms_avg": ms / K,
+                "tflops": p.flops / (ms / K * 1e-3) / 1e12, "replays": reps}
+    except Exception as e:  # noqa: BLE001 - context only
+        return {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
 
 
 def roofline_of(p, gemm_ms, clocks, window_ms, workload_key, kernel_desc):
@@ -675,6 +715,7 @@ def run_ours(args):
                  "kernel_tflops": q.flops / (mq["gemm_ms"] * 1e-3) / 1e12,
                  "roofline": roofline_of(q, mq["gemm_ms"], mq["clocks"], mq["window_ms"], name, mq["kernel_desc"]),
                  "replays": mq["replays"], "window_ms": mq["window_ms"],
+                 "library_context": mq["library"],
                  "clocks": {k: mq["clocks"][k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
                  "device_error": mq["device_error"]}
         if not args.no_cpu_baseline:
