@@ -210,8 +210,9 @@ static Config make_config() {
   c.bn = BN;
   c.stages = STAGES;
   c.ctas = CTAS;
-  c.smem = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED>::kSmemBytes;
-  c.num_acc = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED>::kNumAcc;
+  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED, MODE == MODE_CONTIG && CTAS == 2>;
+  c.smem = L::kSmemBytes;
+  c.num_acc = L::kNumAcc;
   c.pipes = PIPES;
   c.layout = LAYOUT;
   c.splitk = SPLITK;
@@ -315,10 +316,10 @@ struct CostParams {
 // the 1-CTA 224-wide tile, which loads twice the B bytes of a 2-CTA tile per
 // SM; its kb_ns are fitted on that workload (interleaved runs), tile_ns kept.
 // The 256-wide tile has one accumulator, which its epilogue releases as soon
-// as it has been read: its tile_ns is that of the interleaved runs.
+// as it has been read; the 2-CTA tiles pair blocks within each expert's run.
 static const CostParams kCostContig[] = {
-    {128, 1, 1, false, 363, 757}, {224, 1, 1, false, 531, 1345}, {256, 1, 1, false, 517, 2250},
-    {224, 2, 2, false, 434, 2023},
+    {128, 1, 1, false, 363, 757}, {224, 1, 1, false, 531, 1345}, {256, 1, 1, false, 522, 2250},
+    {224, 2, 2, false, 405, 2023},
 };
 static const CostParams kCost[] = {
     {128, 1, 1, false, 360, 757},  {224, 1, 1, false, 453, 1345}, {256, 1, 1, false, 514, 2566},
@@ -355,7 +356,8 @@ static double config_cost(const Config& c, long long rows_est, int N, int K, int
     m_tiles = static_cast<long long>(groups) * ((per + tile_m - 1) / tile_m);
   } else {
     m_tiles = (rows_est + tile_m - 1) / tile_m;
-    if (MODE == MODE_CONTIG && c.ctas == 2) m_tiles += groups;  // second-pass pairs at expert boundaries
+    // pairs within each expert's run of blocks: about one half-empty pair per two experts
+    if (MODE == MODE_CONTIG && c.ctas == 2) m_tiles += (groups + 1) / 2;
   }
   // the last N tile runs a narrower MMA when it is ragged (64 or 128 columns)
   const int full = N / c.bn, rem = N - full * c.bn;
@@ -381,7 +383,8 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms, in
   // A forced tile applies to the entry points that have it built; the others
   // keep the heuristic (each layout and output type builds its own set).
   if (t_force_bn) {
-    if (const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes)) return f;
+    const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes);
+    if (f && !(MODE == MODE_CONTIG && f->ctas == 2 && rows_est / 128 > kMaxContigBlocks)) return f;
   }
   int n = 0;
   const Config* t = config_table<MODE>(&n);
@@ -391,6 +394,8 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms, in
     const Config& c = t[i];
     // split-K tiles keep no second accumulator for overlap; they need at least two groups of 4 K blocks
     if (c.splitk && K <= 4 * 128) continue;
+    // contiguous CTA pairs: the device-built pair table holds kMaxContigBlocks blocks
+    if (MODE == MODE_CONTIG && c.ctas == 2 && rows_est / 128 > kMaxContigBlocks) continue;
     const double cost = config_cost<MODE == MODE_CONTIG || MODE == MODE_MASKED ? MODE : MODE_DENSE>(
         c, rows_est, N, K, sms, groups);
     if (cost < best_cost * 0.999) {
@@ -944,7 +949,8 @@ static int contiguous_impl(const void* a, const void* sfa, const void* b, const 
   args.N = N;
   args.K = K;
   args.G = num_groups;
-  args.num_m_blocks = (M_total + 128 * cfg->ctas - 1) / (128 * cfg->ctas);  // 128-row blocks or block pairs
+  // 128-row blocks (1-CTA tiles) or an estimate of the pairs (2-CTA tiles: the kernel pairs blocks itself)
+  args.num_m_blocks = (M_total + 128 * cfg->ctas - 1) / (128 * cfg->ctas);
   args.num_n_blocks = (N + cfg->bn - 1) / cfg->bn;
   args.raster_m = raster_group(args.num_m_blocks);
   args.m_indices = m_indices;

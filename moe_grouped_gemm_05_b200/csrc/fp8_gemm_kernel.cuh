@@ -87,6 +87,10 @@ template <int PIPES>
 constexpr int kThreadsFor = 32 * (8 + 3 * PIPES);
 constexpr int kThreads = kThreadsFor<1>;
 constexpr int kMaxMaskedGroups = 512;
+// Contiguous layout on CTA pairs: the 128-row blocks are paired within each
+// expert's run of blocks by a table built on the device, for up to this many
+// blocks (M_total <= 131072 rows); the host uses 1-CTA tiles beyond.
+constexpr int kMaxContigBlocks = 1024;
 constexpr int kMaxSmem = 232448;                  // opt-in shared memory per block on sm_100
 // Default limit of every pipeline wait: 2 s, far above any legitimate wait.
 // The main-loop waits take theirs from GemmArgs::wait_limit_ns (this value
@@ -116,7 +120,7 @@ struct GemmArgs {
   uint64_t wait_limit_ns;  // limit of each main-loop wait before the CTA gives up
 };
 
-template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0, bool MASKED = true>
+template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0, bool MASKED = true, bool CPAIRS = false>
 struct Layout {
   static_assert(!(LAYOUT & 2) || (BN / CTAS) % 128 == 0, "an MN-major B tile is whole 128-column boxes per CTA");
   static_assert(CTAS == 1 || CTAS == 2, "CTAS is 1 or 2");
@@ -148,8 +152,10 @@ struct Layout {
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + STAGES * kABytes;
   static constexpr int kOffSft = kOffB + STAGES * kBBytes;
-  // the masked layout's per-expert prefix and counts (other modes keep none)
-  static constexpr int kGroupsBytes = MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : 0;
+  // the masked layout's per-expert prefix and counts; the contiguous layout's
+  // pair table on CTA pairs (count, then first blocks); other modes keep none
+  static constexpr int kGroupsBytes =
+      MASKED ? (2 * kMaxMaskedGroups + 1) * 4 : (CPAIRS ? (kMaxContigBlocks + 1) * 4 : 0);
   // scale ring depth (per pipeline): 4 groups when shared memory allows, else 2
   static constexpr int kSfRing =
       (kOffSft + PIPES * 4 * kSftBytes + 1023) / 1024 * 1024 + 8 * kEpiBuf + 4096 + kGroupsBytes + 1024 <= kMaxSmem
@@ -159,7 +165,7 @@ struct Layout {
   static constexpr int kOffBar = kOffEpi + 8 * kEpiBuf;  // one staging buffer per epilogue warp
   static constexpr int kNumBars = 2 * STAGES + 2 * 2 + 2 + 2 * PIPES * 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;  // tmem addr, abort flag, 2 peer load counts
-  static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]
+  static constexpr int kOffGroups = kOffMisc + 16;          // masked: prefix[G+1], count[G]; contiguous pairs
   static constexpr int kSmemBytes = kOffGroups + kGroupsBytes + 1024;
   static_assert(kSmemBytes <= kMaxSmem, "shared-memory budget exceeded");
   static_assert(kSfBaseCol + PIPES * 2 * kSfSlotCols <= kTmemCols, "TMEM budget exceeded");
@@ -167,6 +173,7 @@ struct Layout {
 
 struct Tile {
   int m_blk, n_blk, g;
+  int row0;  // first row of the tile in A / D (per expert for masked)
 };
 
 // UE8M0 byte of an fp32 scale: the exponent field of a positive normal power
@@ -234,26 +241,32 @@ __device__ __forceinline__ void wait_phase_drain(uint64_t* bar, uint32_t parity)
 template <int MODE, int CTAS>
 __device__ __forceinline__ int total_tiles(const GemmArgs& p, const int* prefix) {
   if (MODE == MODE_MASKED) return prefix[p.G];
-  // contiguous pairs: a second pass for the pairs whose two blocks have different experts
-  if (MODE == MODE_CONTIG && CTAS == 2) return 2 * p.num_m_blocks * p.num_n_blocks;
+  if (MODE == MODE_CONTIG && CTAS == 2) return prefix[0] * p.num_n_blocks;  // pairs from the table
   return p.num_m_blocks * p.num_n_blocks;
 }
 
 // Tile order: dense / contiguous use groups of `raster_m` M blocks swept
 // column by column, so concurrently running CTAs share A rows and B columns
 // in L2; masked runs expert by expert, N block by N block, M blocks fastest.
-// Contiguous 2-CTA tiles pair the 128-row blocks 2j and 2j+1: the first pass
-// (g = 0) computes pair j with the expert of block 2j, the second (g = 1)
-// only the pairs whose block 2j+1 has another expert, with that expert.
+// Contiguous 2-CTA tiles take their M units from the pair table: pairs of
+// consecutive 128-row blocks of one expert's run, a run of odd length ending
+// in a block on its own (the pair's second CTA then stores nothing).
 template <int MODE, int TILE_M>
 __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* prefix,
                                         const int* counts) {
   Tile tl;
-  int pass = 0;
   if (MODE == MODE_CONTIG && TILE_M == 256) {
-    const int per_pass = p.num_m_blocks * p.num_n_blocks;
-    pass = t >= per_pass ? 1 : 0;
-    t -= pass * per_pass;
+    const int pairs = prefix[0];
+    const int per_group = p.raster_m * p.num_n_blocks;
+    const int grp = t / per_group;
+    const int first = grp * p.raster_m;
+    const int gsize = min(p.raster_m, pairs - first);
+    const int within = t - grp * per_group;
+    tl.m_blk = first + within % gsize;
+    tl.n_blk = within / gsize;
+    tl.g = 0;
+    tl.row0 = prefix[1 + tl.m_blk] * 128;
+    return tl;
   }
   if (MODE == MODE_MASKED) {
     int g = 0;
@@ -271,8 +284,9 @@ __device__ __forceinline__ Tile tile_of(int t, const GemmArgs& p, const int* pre
     const int within = t - grp * per_group;
     tl.m_blk = first_m + within % gsize;
     tl.n_blk = within / gsize;
-    tl.g = pass;
+    tl.g = 0;
   }
+  tl.row0 = tl.m_blk * TILE_M;
   return tl;
 }
 
@@ -292,16 +306,13 @@ __device__ __forceinline__ int tile_mma_n(int n0, int N) {
 }
 
 // Expert of a contiguous-layout tile, or -1 when the tile has nothing to
-// compute: its (first) block starts with a padding row or an out-of-range
-// index, or it is a second-pass pair whose blocks share one expert.
+// compute: its (first) block starts with a padding row or an out-of-range index.
 template <int CTAS>
 __device__ __forceinline__ int contig_expert(const Tile& tl, const GemmArgs& p) {
-  const int blocks = p.rows / 128;
-  const int blk = CTAS * tl.m_blk + tl.g;
-  if (blk >= blocks) return -1;
+  const int blk = tl.row0 / 128;
+  if (blk >= p.rows / 128) return -1;
   const int e = __ldg(&p.m_indices[blk * 128]);
   if (e < 0 || e >= p.G) return -1;
-  if (CTAS == 2 && tl.g == 1 && __ldg(&p.m_indices[(blk - 1) * 128]) == e) return -1;
   return e;
 }
 
@@ -310,7 +321,7 @@ template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPE
 __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
-  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED>;
+  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED, MODE == MODE_CONTIG && CTAS == 2>;
   static_assert(LAYOUT == 0 || MODE == MODE_DENSE, "MN-major operands are built for the dense GEMM only");
   static_assert(!SPLITK || PIPES == 2, "split-K runs on two pipelines");
   constexpr bool kAmn = (LAYOUT & 1) != 0;
@@ -411,6 +422,44 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     }
     if (lane == 0) prefix[0] = 0;
   }
+  if (MODE == MODE_CONTIG && kPair && warp == kEpi0) {
+    // Pair table: block b (128 rows, expert = that of its first row) starts a
+    // pair when it lies an even number of blocks into its run of equal
+    // experts; blocks with an index outside [0, G) start none.  The experts
+    // of all blocks are loaded at once (at most 32 per lane), then scanned.
+    const int nb = p.rows / 128;
+    int ev[kMaxContigBlocks / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxContigBlocks / 32; ++i) {
+      const int b = 32 * i + lane;
+      ev[i] = b < nb ? __ldg(&p.m_indices[b * 128]) : -1;
+    }
+    int count = 0, run_start = 0, prev_e = -2;
+#pragma unroll
+    for (int i = 0; i < kMaxContigBlocks / 32; ++i) {
+      if (32 * i >= nb) break;
+      const int b = 32 * i + lane;
+      const int e = ev[i];
+      if (b < nb && (e < -1 || e >= p.G) && blockIdx.x == 0) atomicOr(&g_dg_error, 0x2);
+      int e_prev = __shfl_up_sync(0xffffffffu, e, 1);
+      if (lane == 0) e_prev = prev_e;
+      // start of the run holding block b: the last block <= b where the expert changes
+      int rs = (b < nb && (b == 0 || e != e_prev)) ? b : -1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, rs, o);
+        if (lane >= o) rs = max(rs, v);
+      }
+      if (rs < 0) rs = run_start;
+      const bool starts = b < nb && e >= 0 && e < p.G && ((b - rs) & 1) == 0;
+      const uint32_t bal = __ballot_sync(0xffffffffu, starts);
+      if (starts) prefix[1 + count + __popc(bal & ((1u << lane) - 1u))] = b;
+      count += __popc(bal);
+      run_start = __shfl_sync(0xffffffffu, rs, 31);
+      prev_e = __shfl_sync(0xffffffffu, e, 31);
+    }
+    if (lane == 0) prefix[0] = count;
+  }
   tc_fence_before();
   if constexpr (kPair) cluster_sync(); else __syncthreads();
   tc_fence_after();
@@ -459,7 +508,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       }
       int gb, ge;
       if (!plan(li, gb, ge)) continue;
-      const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
+      const int m_base = tl.row0 + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
       const int kb_hi = min(num_kb, 4 * ge);
       for (int kb = 4 * gb; kb < kb_hi; ++kb, ++it) {
@@ -644,7 +693,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       }
       int gb, ge;
       if (!plan(li, gb, ge)) continue;
-      const int m_base = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank);
+      const int m_base = tl.row0 + 128 * static_cast<int>(rank);
       const int n0 = tl.n_blk * BN;
       for (int kp = gb; kp < ge; ++kp, ++group) {
         const uint32_t ring = group % L::kSfRing;
@@ -724,9 +773,9 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       int expert = 0, own_e = 0;
       if (MODE == MODE_CONTIG) {
         // expert of this CTA's own 128-row block (a pair's blocks may differ)
-        const int own_blk = CTAS * tl.m_blk + static_cast<int>(rank);
+        const int own_blk = tl.row0 / 128 + static_cast<int>(rank);
         own_e = own_blk < p.rows / 128 ? __ldg(&p.m_indices[own_blk * 128]) : -1;
-        if ((own_e < -1 || own_e >= p.G) && warp == kEpi0 && lane == 0 && tl.n_blk == 0 && tl.g == 0)
+        if ((own_e < -1 || own_e >= p.G) && warp == kEpi0 && lane == 0 && tl.n_blk == 0)
           atomicOr(&g_dg_error, 0x2);
         expert = contig_expert<CTAS>(tl, p);
         if (expert < 0) continue;
@@ -749,7 +798,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       if (!ok) break;
       tc_fence_after();
 
-      const int row0 = tl.m_blk * L::kTileM + 128 * static_cast<int>(rank) + 32 * q;  // warp's first row
+      const int row0 = tl.row0 + 128 * static_cast<int>(rank) + 32 * q;  // warp's first row
       const int m_local = row0 + lane;  // row inside A / D (per expert for masked)
       bool valid;
       if (MODE == MODE_DENSE) {

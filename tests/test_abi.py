@@ -124,7 +124,9 @@ def test_heuristic_choices_without_gpu(lib):
     assert dg.describe_config("dense", 64, 7168, 512) == "128x64x8/112"  # one K group: no split
     masked = dg.describe_config("masked", 256, 7168, 2048, 16)
     assert "(2cta)" not in masked and masked.startswith("128x")
-    assert dg.describe_config("contiguous", 32768, 4096, 7168, 8) == "128x256x4/148"
+    assert dg.describe_config("contiguous", 32768, 4096, 7168, 8) == "256x224x6(2cta)(2pipe)/148"
+    # beyond the pair table's 1024 blocks the contiguous layout keeps 1-CTA tiles
+    assert "(2cta)" not in dg.describe_config("contiguous", 1024 * 128 + 128, 4096, 7168, 8)
 
 
 def test_tc_util_caps_the_planned_grid(lib):

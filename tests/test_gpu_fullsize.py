@@ -68,24 +68,32 @@ def test_dense_full_size(name):
 
 
 def test_contiguous_full_size():
+    """The heuristic's configuration and the 2-CTA tiles whose block pairs the
+    kernel forms within each expert's run, both against one oracle result."""
     p = synth.WORKLOADS["contiguous_8x4096x7168_zipf1.1"]()
     sfa, sa = _pack_on_gpu(p.sfa)
     sfb, sb = _pack_on_gpu(p.sfb)
-    d = _sentinel((p.M, p.N))
-    dg.m_grouped_fp8_gemm_nt_contiguous(_fp8(p.a), sfa, _fp8(p.b), sfb, torch.from_numpy(p.m_indices).cuda(), d)
-    torch.cuda.synchronize()
-    assert dg.get_device_error() == 0
-    got = bits(d)
     pad = p.m_indices < 0
-    assert (got[pad] == SENTINEL).all(), "padding rows were written"
-    ref = np.full_like(got, SENTINEL)
+    ref = np.full((p.M, p.N), SENTINEL, np.uint16)
     for e in range(p.G):
         rows = np.nonzero(p.m_indices == e)[0]
         assert len(rows) > 0
         ref[rows] = oracle_rows(p.a, sa, p.b[e], sb[e], p.M, p.N, p.K, rows)
-        check_close(got[rows], ref[rows], f"contiguous expert {e}")
-    # the whole call's normalised difference, over every valid row
-    check_close(got[~pad], ref[~pad], "contiguous, all valid rows")
+    a, b, mi = _fp8(p.a), _fp8(p.b), torch.from_numpy(p.m_indices).cuda()
+    for cfg in ((0, 0, 0), (224, 2, 2)):
+        dg.set_config(*cfg)
+        d = _sentinel((p.M, p.N))
+        dg.m_grouped_fp8_gemm_nt_contiguous(a, sfa, b, sfb, mi, d)
+        torch.cuda.synchronize()
+        dg.set_config(0)
+        assert dg.get_device_error() == 0
+        got = bits(d)
+        assert (got[pad] == SENTINEL).all(), f"padding rows were written, cfg={cfg}"
+        for e in range(p.G):
+            rows = np.nonzero(p.m_indices == e)[0]
+            check_close(got[rows], ref[rows], f"contiguous expert {e}, cfg={cfg}")
+        # the whole call's normalised difference, over every valid row
+        check_close(got[~pad], ref[~pad], f"contiguous, all valid rows, cfg={cfg}")
 
 
 def test_masked_full_size():
