@@ -8,7 +8,7 @@ import oracle
 from moe_grouped_gemm_05_b200 import binding as dg
 from moe_grouped_gemm_05_b200 import synth
 
-from helpers import bits, check_close, packed, to_device
+from helpers import bits, check_close, oracle_rows, packed, to_device
 
 pytestmark = pytest.mark.gpu
 SENTINEL = 0xDEAD
@@ -108,4 +108,41 @@ def test_contiguous_many_small_experts():
         got = bits(d)
         check_close(got[valid], ref[valid], f"many experts cfg={cfg}")
         assert (got[~valid] == SENTINEL).all()
+    assert dg.get_device_error() == 0
+
+
+def test_contiguous_pair_table_at_its_maximum():
+    """1024 blocks of 128 rows (131072 rows, the most the 2-CTA tiles' pair
+    table holds), 32 experts of 32 blocks each with ragged last blocks."""
+    rng = np.random.default_rng(504)
+    counts = 32 * 128 - rng.integers(0, 128, 32)
+    p = synth.contiguous_problem(32, 256, 128, rows=0, seed=504, counts=list(counts))
+    assert p.M == 1024 * 128
+    sa, sb = packed(p)
+    t = to_device(p, sa, sb)
+    valid = p.m_indices >= 0
+    ref = np.full((p.M, p.N), SENTINEL, np.uint16)
+    for e in range(p.G):
+        rows = np.nonzero(p.m_indices == e)[0]
+        ref[rows] = oracle_rows(p.a, sa, p.b[e], sb[e], p.M, p.N, p.K, rows)
+    dg.set_config(224, 2, 2)
+    assert "(2cta)" in dg.describe_config("contiguous", p.M, p.N, p.K, p.G)
+    d = _sentinel((p.M, p.N))
+    dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], t["m_indices"], d)
+    got = bits(d)
+    check_close(got[valid], ref[valid], "pair table with 1024 blocks")
+    assert (got[~valid] == SENTINEL).all()
+    assert dg.get_device_error() == 0
+
+
+@pytest.mark.parametrize("cfg", [(0, 0, 0), (224, 2, 2)])
+def test_contiguous_all_padding_writes_nothing(cfg):
+    p = synth.contiguous_problem(3, 256, 256, rows=0, seed=505, counts=[128, 128, 128])
+    sa, sb = packed(p)
+    t = to_device(p, sa, sb)
+    t["m_indices"] = torch.full((p.M,), -1, dtype=torch.int32, device="cuda")
+    dg.set_config(*cfg)
+    d = _sentinel((p.M, p.N))
+    dg.m_grouped_fp8_gemm_nt_contiguous(t["a"], t["sfa"], t["b"], t["sfb"], t["m_indices"], d)
+    assert (bits(d) == SENTINEL).all()
     assert dg.get_device_error() == 0

@@ -197,7 +197,9 @@ def test_contiguous_block_pairs_edge_layouts(cfg):
     assert dg.get_device_error() == 0
 
 
-def test_contiguous_bad_expert_index_flags_and_skips():
+@pytest.mark.parametrize("cfg", BUILT_CONTIG)
+def test_contiguous_bad_expert_index_flags_and_skips(cfg):
+    dg.set_config(*cfg)
     p = synth.contiguous_problem(2, 256, 256, rows=0, seed=78, counts=[128, 100])
     sa, sb = packed(p)
     idx = p.m_indices.copy()
