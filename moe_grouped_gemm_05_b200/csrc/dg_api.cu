@@ -199,32 +199,34 @@ struct Config {
   int pipes = 1;  // load/MMA pipelines per CTA (alternate tiles)
   int layout = 0; // bit 0: A MN-major, bit 1: B MN-major
   bool splitk = false;  // both pipelines on every tile, each on half of K
+  int a_rows = 128;     // rows of A per stage and TMA box: 128, or 64 for problems of at most 64 rows
   int threads = kThreads;
   KernelFn fn = nullptr;
 };
 
 template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0,
-          bool SPLITK = false>
+          bool SPLITK = false, int A_ROWS = 128>
 static Config make_config() {
   Config c;
   c.bn = BN;
   c.stages = STAGES;
   c.ctas = CTAS;
-  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED, MODE == MODE_CONTIG && CTAS == 2>;
+  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED, MODE == MODE_CONTIG && CTAS == 2, A_ROWS>;
   c.smem = L::kSmemBytes;
   c.num_acc = L::kNumAcc;
   c.pipes = PIPES;
   c.layout = LAYOUT;
   c.splitk = SPLITK;
+  c.a_rows = A_ROWS;
   c.threads = kThreadsFor<PIPES>;
-  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES, LAYOUT, SPLITK>);
+  c.fn = reinterpret_cast<KernelFn>(&fp8_gemm_kernel<BN, STAGES, MODE, CTAS, OUT_F32, PIPES, LAYOUT, SPLITK, A_ROWS>);
   return c;
 }
 
 // Built configurations.  A 2-CTA tile spans 256 rows, which the contiguous
 // layout (128-row expert alignment) cannot guarantee to be one expert; its
-// 2-CTA tiles pair blocks 2j and 2j+1 and run a second pass for the pairs
-// that straddle an expert boundary (at most one per expert).
+// 2-CTA tiles pair 128-row blocks within each expert's run of blocks (a table
+// the kernel builds from m_indices), an odd run ending in a half-empty pair.
 // Host-side id of the dense kernels with FP32 output (optionally + C).
 constexpr int MODE_DENSE_F32 = 3;
 // Host-side ids of the dense kernels with MN-major operands: MODE_DENSE_MN + LAYOUT - 1
@@ -268,7 +270,11 @@ static const Config* config_table(int* count) {
         make_config<128, 6, MODE, 1>(), make_config<224, 4, MODE, 1>(), make_config<256, 4, MODE, 1>(),
         make_config<128, 6, MODE, 2>(), make_config<224, 6, MODE, 2>(), make_config<256, 6, MODE, 2>(),
         make_config<224, 6, MODE, 2, false, 2>(), make_config<128, 6, MODE, 2, false, 2>(),
-        make_config<64, 8, MODE, 1>(), make_config<64, (MODE == MODE_DENSE ? 8 : 6), MODE, 1, false, 2, 0, true>(),
+        make_config<64, 8, MODE, 1>(),
+        // decode: split-K tiles with 64-row A stages (problems of at most 64 rows per group) come
+        // first, so that they win ties and forced lookups where they fit
+        make_config<64, (MODE == MODE_DENSE ? 12 : 10), MODE, 1, false, 2, 0, true, 64>(),
+        make_config<64, (MODE == MODE_DENSE ? 8 : 6), MODE, 1, false, 2, 0, true>(),
         make_config<128, 4, MODE, 1, false, 2, 0, true>(),
     };
     *count = static_cast<int>(sizeof(table) / sizeof(table[0]));
@@ -276,14 +282,18 @@ static const Config* config_table(int* count) {
   }
 }
 
+// Whether configuration c can run a problem whose groups hold a_extent rows of A.
+static bool a_rows_fit(const Config& c, long long a_extent) { return c.a_rows == 128 || a_extent <= c.a_rows; }
+
 // First built configuration with this tile width, CTA count (0: any) and
-// number of pipelines (0: any).
+// number of pipelines (0: any) that fits groups of a_extent rows of A (-1: any size).
 template <int MODE>
-static const Config* find_config(int bn, int ctas, int pipes = 0) {
+static const Config* find_config(int bn, int ctas, int pipes = 0, long long a_extent = -1) {
   int n = 0;
   const Config* t = config_table<MODE>(&n);
   for (int i = 0; i < n; ++i)
-    if (t[i].bn == bn && (ctas == 0 || t[i].ctas == ctas) && (pipes == 0 || t[i].pipes == pipes))
+    if (t[i].bn == bn && (ctas == 0 || t[i].ctas == ctas) && (pipes == 0 || t[i].pipes == pipes) &&
+        (a_extent < 0 || a_rows_fit(t[i], a_extent)))
       return &t[i];
   return nullptr;
 }
@@ -378,12 +388,15 @@ static double config_cost(const Config& c, long long rows_est, int N, int K, int
   return std::max(compute, memory) + 0.1 * std::min(compute, memory);
 }
 
+// a_extent: rows of A per group (dense and contiguous: the rows; masked: M_max), -1 for rows_est.
 template <int MODE>
-static const Config* choose_config(long long rows_est, int N, int K, int sms, int groups = 1) {
+static const Config* choose_config(long long rows_est, int N, int K, int sms, int groups = 1,
+                                   long long a_extent = -1) {
+  if (a_extent < 0) a_extent = rows_est;
   // A forced tile applies to the entry points that have it built; the others
   // keep the heuristic (each layout and output type builds its own set).
   if (t_force_bn) {
-    const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes);
+    const Config* f = find_config<MODE>(t_force_bn, t_force_ctas, t_force_pipes, a_extent);
     if (f && !(MODE == MODE_CONTIG && f->ctas == 2 && rows_est / 128 > kMaxContigBlocks)) return f;
   }
   int n = 0;
@@ -392,6 +405,7 @@ static const Config* choose_config(long long rows_est, int N, int K, int sms, in
   double best_cost = 1e300;
   for (int i = 0; i < n; ++i) {
     const Config& c = t[i];
+    if (!a_rows_fit(c, a_extent)) continue;
     // split-K tiles keep no second accumulator for overlap; they need at least two groups of 4 K blocks
     if (c.splitk && K <= 4 * 128) continue;
     // contiguous CTA pairs: the device-built pair table holds kMaxContigBlocks blocks
@@ -478,7 +492,7 @@ static int launch(const Config* cfg, int grid, const CUtensorMap* maps, GemmArgs
 }
 
 // Builds the tensor maps of one call.
-//   A : [GA][rowsA][K] bytes    box 128 x 128 (K x rows), 128-byte swizzle
+//   A : [GA][rowsA][K] bytes    box 128 x 128 (K x rows; 128 x 64 with 64-row stages), 128-byte swizzle
 //       ([GA][K][rowsA] when MN-major: box 128 x 128 (rows x K))
 //   B : [GB][N][K] bytes        box 128 x BN/CTAS,         128-byte swizzle
 //       ([GB][K][N] when MN-major: box 128 x 128 (N x K), BN/CTAS/128 boxes per stage)
@@ -491,7 +505,7 @@ static int build_maps(CUtensorMap* maps, const Config* cfg, const void* a, const
                       static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A")))
       return r;
   } else if ((r = make_map(&maps[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, a, K, rowsA, GA, K,
-                           static_cast<uint64_t>(rowsA) * K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B, "A"))) {
+                           static_cast<uint64_t>(rowsA) * K, 128, cfg->a_rows, CU_TENSOR_MAP_SWIZZLE_128B, "A"))) {
     return r;
   }
   if (cfg->layout & 2) {  // B stored [GB][K][N]: 128 columns x 128 K per box
@@ -735,15 +749,16 @@ int dg_describe_config(int kind, int M, int N, int K, int num_groups, char* buf,
   long long tiles = 0;
   if (kind == 2) {
     const long long est = std::max<long long>(1, static_cast<long long>(num_groups) * M / 2);
-    c = choose_config<MODE_MASKED>(est, N, K, sms, num_groups);
+    c = choose_config<MODE_MASKED>(est, N, K, sms, num_groups, M);
     if (c) tiles = static_cast<long long>(num_groups) * ((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   } else {
     c = kind == 1 ? choose_config<MODE_CONTIG>(M, N, K, sms, num_groups) : choose_config<MODE_DENSE>(M, N, K, sms);
     if (c) tiles = static_cast<long long>((M + 128 * c->ctas - 1) / (128 * c->ctas)) * ((N + c->bn - 1) / c->bn);
   }
   if (!c) return fail(DG_ERR_UNSUPPORTED, "no configuration");
-  snprintf(buf, buflen, "%dx%dx%d%s%s%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
-           c->pipes == 2 ? "(2pipe)" : "", c->splitk ? "(splitk)" : "", grid_size(device_sms, tiles, c));
+  snprintf(buf, buflen, "%dx%dx%d%s%s%s%s/%d", 128 * c->ctas, c->bn, c->stages, c->ctas == 2 ? "(2cta)" : "",
+           c->pipes == 2 ? "(2pipe)" : "", c->splitk ? "(splitk)" : "", c->a_rows == 64 ? "(a64)" : "",
+           grid_size(device_sms, tiles, c));
   return DG_OK;
 }
 
@@ -987,7 +1002,7 @@ static int masked_impl(const void* a, const void* sfa, const void* b, const int3
   if ((r = device_info(&di))) return r;
   // the device decides the real tile count; the heuristic assumes half-full experts
   const long long rows_est = std::max<long long>(1, static_cast<long long>(num_groups) * M_max / 2);
-  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, usable_sms(di.sms), num_groups);
+  const Config* cfg = choose_config<MODE_MASKED>(rows_est, N, K, usable_sms(di.sms), num_groups, M_max);
   if (!cfg) return fail(DG_ERR_UNSUPPORTED, "no built configuration");
   CUtensorMap maps[3];
   if ((r = build_maps_cached(maps, cfg, a, b, d, M_max, num_groups, N, K, num_groups, M_max, num_groups)))

@@ -120,7 +120,8 @@ struct GemmArgs {
   uint64_t wait_limit_ns;  // limit of each main-loop wait before the CTA gives up
 };
 
-template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0, bool MASKED = true, bool CPAIRS = false>
+template <int BN, int STAGES, int CTAS, int PIPES = 1, int LAYOUT = 0, bool MASKED = true, bool CPAIRS = false,
+          int A_ROWS = 128>
 struct Layout {
   static_assert(!(LAYOUT & 2) || (BN / CTAS) % 128 == 0, "an MN-major B tile is whole 128-column boxes per CTA");
   static_assert(CTAS == 1 || CTAS == 2, "CTAS is 1 or 2");
@@ -131,7 +132,14 @@ struct Layout {
   static constexpr int kTileM = 128 * CTAS;
   static constexpr int kBRows = BN / CTAS;              // rows of B loaded by each CTA
   static constexpr int kNB128 = (BN + 127) / 128;       // 128-column groups of B scales
-  static constexpr int kABytes = 128 * kBK;             // 16 KB
+  // Rows of A per stage: 128, or 64 for problems of at most 64 rows (A
+  // K-major, 1-CTA tiles).  The MMA stays 128 rows tall; with 64-row stages
+  // its rows 64-127 read the next 8 KB of shared memory (the next stage, or
+  // the first B stage), so those accumulator rows hold garbage that no store
+  // writes out (they are rows >= M), and each stage takes a third less room.
+  static_assert(A_ROWS == 128 || (A_ROWS == 64 && CTAS == 1 && (LAYOUT & 1) == 0),
+                "64-row A stages are built for K-major A on 1-CTA tiles");
+  static constexpr int kABytes = A_ROWS * kBK;          // 16 KB (8 KB with 64-row stages)
   static constexpr int kBBytes = kBRows * kBK;
   // Scale words of one K group in shared memory, as tcgen05.cp sources:
   // 128 rows x 32 B (core-matrix layout) holding [SFA | SFB of columns 0-127]
@@ -317,11 +325,12 @@ __device__ __forceinline__ int contig_expert(const Tile& tl, const GemmArgs& p) 
 }
 
 template <int BN, int STAGES, int MODE, int CTAS, bool OUT_F32 = false, int PIPES = 1, int LAYOUT = 0,
-          bool SPLITK = false>
+          bool SPLITK = false, int A_ROWS = 128>
 __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                     const __grid_constant__ CUtensorMap tm_d, const GemmArgs p) {
-  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED, MODE == MODE_CONTIG && CTAS == 2>;
+  using L = Layout<BN, STAGES, CTAS, PIPES, LAYOUT, MODE == MODE_MASKED, MODE == MODE_CONTIG && CTAS == 2, A_ROWS>;
+  static_assert(A_ROWS == 128 || MODE != MODE_CONTIG, "64-row A stages hold one tile's rows: dense and masked only");
   static_assert(LAYOUT == 0 || MODE == MODE_DENSE, "MN-major operands are built for the dense GEMM only");
   static_assert(!SPLITK || PIPES == 2, "split-K runs on two pipelines");
   constexpr bool kAmn = (LAYOUT & 1) != 0;

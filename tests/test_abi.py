@@ -118,7 +118,18 @@ def test_heuristic_choices_without_gpu(lib):
     1-CTA tiles, and the pick is stable for the workloads the bench times."""
     from moe_grouped_gemm_05_b200 import binding as dg
 
-    assert dg.describe_config("dense", 64, 7168, 2048).startswith("128x64x8(2pipe)(splitk)/112")
+    # at most 64 rows: split-K tiles whose stages hold 64 rows of A
+    assert dg.describe_config("dense", 64, 7168, 2048) == "128x64x12(2pipe)(splitk)(a64)/112"
+    assert dg.describe_config("dense", 1, 7168, 2048) == "128x64x12(2pipe)(splitk)(a64)/112"
+    assert dg.describe_config("dense", 65, 7168, 2048) == "128x64x8(2pipe)(splitk)/112"
+    assert dg.describe_config("masked", 64, 256, 2048, 4) == "128x64x10(2pipe)(splitk)(a64)/16"
+    assert dg.describe_config("masked", 65, 256, 2048, 4) == "128x64x6(2pipe)(splitk)/16"
+    assert lib.dg_set_config(64, 1, 2) == 0  # a forced tile takes the 64-row stages where they fit
+    try:
+        assert dg.describe_config("dense", 64, 464, 2048).endswith("(a64)/8")
+        assert "(a64)" not in dg.describe_config("dense", 65, 464, 2048)
+    finally:
+        assert lib.dg_set_config(0, 0, 0) == 0
     assert dg.describe_config("dense", 4096, 7168, 2048) == "256x224x6(2cta)(2pipe)/148"
     assert dg.describe_config("dense", 8192, 8192, 8192) == "256x224x6(2cta)(2pipe)/148"
     assert dg.describe_config("dense", 64, 7168, 512) == "128x64x8/112"  # one K group: no split
