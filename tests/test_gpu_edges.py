@@ -92,7 +92,8 @@ def test_masked_largest_group_count():
 
 
 def test_contiguous_many_small_experts():
-    """64 experts with 0-200 rows each: many segments, many block pairs straddling experts."""
+    """64 experts with 0-200 rows each: many short segments, empty experts, and
+    runs of one or two blocks (half-empty CTA pairs on the 2-CTA tiles)."""
     rng = np.random.default_rng(503)
     counts = rng.integers(0, 201, 64)
     p = synth.contiguous_problem(64, 256, 384, rows=0, seed=503, counts=list(counts))
