@@ -17,11 +17,14 @@ Zipf-routed rows, N=4096, K=7168); with one GPU the same line carries a
 ``workloads`` object with every workload measured in the same run (kernel
 configuration, time, TFLOPS, roofline fraction and the CPU oracle's rate).
 
-With N > 1 (torchrun, one process per GPU) the headline problem is split
-across the ranks along N in whole 128-column blocks (each rank holds A, its
-slice of every expert's weights and its columns of D; ``--shard experts``
-splits the experts instead): strong scaling, no collective on the data path,
-time = max over ranks.
+With N > 1 (torchrun, one process per GPU) the ranks share one problem
+with no collective on the data path; time = max over ranks.  By default
+(weak scaling) the problem grows with the ranks: it is the headline problem
+widened P-fold along N, each rank owning an N-column block of every
+expert's weights and of D (``--shard experts``: P times the experts, each
+rank owning the headline's experts and their routed rows), so every rank
+runs the headline shape.  ``--scaling strong`` splits the headline problem
+itself instead (N in whole 128-column blocks, or the experts).
 """
 from __future__ import annotations
 
@@ -61,6 +64,9 @@ def parse_args():
                     help="workloads measured into the line's 'workloads' object at N=1: all, none or a comma list")
     ap.add_argument("--shard", choices=["n", "experts"], default="n",
                     help="N > 1: split N across ranks (default) or, for grouped workloads, the experts")
+    ap.add_argument("--scaling", choices=["weak", "strong"], default="weak",
+                    help="N > 1: each rank owns a headline-sized share of a P-times larger problem (weak), "
+                         "or a 1/P share of the headline problem (strong)")
     ap.add_argument("--min-window-ms", type=float, default=200.0,
                     help="each timing is repeated (K-step graph replays) until this much device time is covered")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -347,6 +353,24 @@ def run_reference(args):
             "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def global_problem(p, world: int, how: str) -> dict:
+    """The whole job's problem under weak scaling: `p` (the headline problem)
+    is every rank's share of a problem P times larger along N ("n") or in
+    experts and their routed rows ("experts", grouped problems)."""
+    g = {"kind": p.kind, "M": p.M, "N": p.N, "K": p.K, "G": p.G, "valid_rows": p.valid_rows}
+    if world > 1:
+        if how == "experts" and p.kind != "dense":
+            g["G"] = p.G * world
+            if p.kind == "contiguous":
+                g["M"], g["valid_rows"] = p.M * world, p.valid_rows * world
+            else:
+                g["valid_rows"] = p.valid_rows * world
+        else:
+            g["N"] = p.N * world
+    g["flops"] = p.flops * world
+    return g
 
 
 def shard_problem(p, world: int, rank: int, how: str):
@@ -649,31 +673,36 @@ def run_ours(args):
 
     lib = dg.load()
     full = synth.WORKLOADS[args.workload]()
-    p = shard_problem(full, world, rank, args.shard)
+    weak = args.scaling == "weak"
+    # weak: every rank runs the headline shape as its share; strong: a 1/P share of it
+    p = full if weak else shard_problem(full, world, rank, args.shard)
+    job = global_problem(full, world, args.shard) if weak else global_problem(full, 1, args.shard)
     m = measure(p, dg, lib, torch, args, dev, local, barrier)
     e2e = None if args.no_e2e else e2e_loop(p, m, dg, lib, torch, args, barrier)
     m["sets"] = None
     torch.cuda.empty_cache()
 
-    # max over ranks of every time; the work is the whole (unsharded) problem's
+    # max over ranks of every time; the work is the whole job's problem
     step_ms = shard.max_over_ranks(m["step_ms"])
     gemm_ms = shard.max_over_ranks(m["gemm_ms"])
     e2e_ms = shard.max_over_ranks(e2e["ms"]) if e2e else None
-    flops = full.flops
+    flops = job["flops"]
     value = flops / (step_ms * 1e-3) / 1e12
     # roofline of this rank's kernel on this rank's share (rank 0 reports it)
-    roof = roofline_of(p, m["gemm_ms"], m["clocks"], m["window_ms"], args.workload if world == 1 else p.name,
-                       m["kernel_desc"])
+    roof = roofline_of(p, m["gemm_ms"], m["clocks"], m["window_ms"],
+                       args.workload if (world == 1 or weak) else p.name, m["kernel_desc"])
     clocks = m["clocks"]
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True,
-        "scaling": "strong" if world > 1 else "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "scaling": "weak" if (weak or world == 1) else "strong", "vs_baseline": None, "dtype": "fp8_e4m3",
         "data": "synthetic",
         "config": {"workload": args.workload, "kind": full.kind, "M": full.M, "N": full.N, "K": full.K, "G": full.G,
                    "valid_rows": full.valid_rows, "kernel_config": m["kernel_desc"],
-                   "parallelism": (f"{world} ranks, " + ("N split in 128-column blocks" if args.shard == "n"
-                                                         or full.kind == "dense" else "experts split")
+                   "parallelism": (f"{world} ranks, " + ("N split" if args.shard == "n" or full.kind == "dense"
+                                                         else "experts split")
+                                   + (f", each rank owning a {full.name} share of a {world}x larger problem"
+                                      if weak else " of the headline problem in 128-column blocks / expert sets")
                                    if world > 1 else "one GPU"),
                    "step": ("GEMM reading A's fp32 scales, packed to UE8M0 in its scale-producer warp"
                             if args.fused_pack else "pack activation scales (fp32 -> UE8M0 int32) + GEMM"),
@@ -689,6 +718,10 @@ def run_ours(args):
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "device_error": m["device_error"],
     }
+    if world > 1:
+        # the whole job's problem; with weak scaling every rank's share holds the headline problem's values
+        line["config"]["job_problem"] = {k: v for k, v in job.items() if k != "flops"}
+        line["config"]["job_flop"] = job["flops"]
     if e2e:
         line["e2e"] = {"value": flops * e2e["steps"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],

@@ -103,3 +103,26 @@ def test_shard_problem_experts_keeps_every_valid_row_once():
             assert len(j) >= 1 and p.m_indices[j[0]] >= 0
         seen.append(int(valid.sum()))
     assert sum(seen) == p.valid_rows
+
+
+def test_weak_scaling_job_problem():
+    """Weak scaling: P ranks each own a headline-sized share of a problem P
+    times larger (along N, or in experts and their routed rows); the job's
+    FLOP are P times the headline's, and one rank is the headline itself."""
+    from moe_grouped_gemm_05_b200 import synth
+
+    p = _contig_problem()
+    one = bench.global_problem(p, 1, "n")
+    assert (one["N"], one["G"], one["M"], one["flops"]) == (p.N, p.G, p.M, p.flops)
+    g = bench.global_problem(p, 4, "n")
+    assert (g["N"], g["G"], g["M"]) == (4 * p.N, p.G, p.M) and g["flops"] == 4 * p.flops
+    # N-split shares of the job problem are each the headline's N columns
+    assert g["N"] // 4 == p.N
+    e = bench.global_problem(p, 4, "experts")
+    assert (e["N"], e["G"], e["M"], e["valid_rows"]) == (p.N, 4 * p.G, 4 * p.M, 4 * p.valid_rows)
+    assert e["flops"] == 4 * p.flops
+    d = synth.dense_problem(64, 256, 256, seed=4)
+    assert bench.global_problem(d, 2, "experts")["N"] == 2 * d.N  # dense problems always split N
+    m = synth.masked_problem(3, 128, 256, 256, seed=5)
+    mg = bench.global_problem(m, 2, "experts")
+    assert (mg["G"], mg["M"], mg["valid_rows"]) == (6, m.M, 2 * m.valid_rows)
