@@ -70,6 +70,9 @@ def parse_args():
     ap.add_argument("--min-window-ms", type=float, default=200.0,
                     help="each timing is repeated (K-step graph replays) until this much device time is covered")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the next-row measurements (quantisation, MoE permute/combine, layouts, FP32 + C, 1D1D)")
+    ap.add_argument("--next-cpu-seconds", type=float, default=1.5, help="oracle time of each next row's CPU sample")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="target CPU time of the headline's oracle sample")
     ap.add_argument("--e2e-steps", type=int, default=0, help="steps of the end-to-end loop (0 = min(steps, 100))")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end loop (profiling runs)")
@@ -563,6 +566,240 @@ def roofline_of(p, gemm_ms, clocks, window_ms, workload_key, kernel_desc):
             + " per launch"}
 
 
+# ---------------------------------------------------------------- the "next" rows
+
+# The MoE step around the contiguous GEMM: 16384 tokens routed top-2 over 8
+# experts (Zipf(1.1) weights), hidden K = 7168, expert output N = 4096.
+NEXT_T, NEXT_TOPK, NEXT_G, NEXT_K, NEXT_N = 16384, 2, 8, 7168, 4096
+
+
+def _graph_time(fn, torch, args, local):
+    """Median device time (ms) of one launch of fn(i): K launches captured in a
+    CUDA graph, replayed until --min-window-ms of device time is covered, with
+    the clocks sampled meanwhile.  Returns (ms, replays, window_ms, clocks)."""
+    K = args.steps
+    for i in range(3):
+        fn(i)
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(cap):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            for i in range(K):
+                fn(i)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+    ev = []
+    while len(ev) < 3 or (sum(ev) < args.min_window_ms and len(ev) < 5000):
+        pairs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(max(1, min(64, len(ev) + 1)))]
+        for a, b in pairs:
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ev += [a.elapsed_time(b) for a, b in pairs]
+    sampler.stop()
+    del g
+    return statistics.median(ev) / K, len(ev), sum(ev), sampler.summary()
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        return os.cpu_count() or 1
+
+
+def _timed_cpu(fn, seconds: float, unit_fn, sample_fn):
+    """The oracle on a growing sample until one run takes about `seconds`; returns its rate."""
+    n = 1
+    while True:
+        t0 = time.perf_counter()
+        fn(n)
+        t = time.perf_counter() - t0
+        if t >= 0.25 * seconds or n >= sample_fn(None):
+            break
+        n = min(sample_fn(None), n * 4)
+    n = int(max(1, min(sample_fn(None), n * seconds / max(t, 1e-6))))
+    t0 = time.perf_counter()
+    fn(n)
+    t = time.perf_counter() - t0
+    value, unit = unit_fn(n, t)
+    return {"value": value, "unit": unit, "cores": int(_cores()), "kind": "oracle", "sample": sample_fn(n) +
+            f", {t:.2f} s per run on host cores"}
+
+
+def _next_row(what, timing, *, flops=None, nbytes=None, cpu=None):
+    """One next-row entry: time, roofline (tensor-bound when the FLOP per byte
+    exceed the ridge, else HBM-bound) and the oracle's rate."""
+    ms, reps, window, clocks = timing
+    peaks, src = load_peaks()
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    long_region = window > 500.0 or capped
+    if flops is not None and (nbytes is None or flops / nbytes > 560.0):
+        peak = 2.0 * peaks.get("bf16_tflops_sustained" if long_region else "bf16_tflops")
+        roof = {"bound": "tensor", "achieved": flops / (ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+                "algorithmic": f"{flops:.4g} FLOP per launch",
+                "peak_source": f"{'sustained' if long_region else 'burst'} bf16 x2 ({src} peaks)"}
+    else:
+        peak = peaks.get("hbm_gbs")
+        roof = {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                "algorithmic": f"{nbytes:.4g} B per launch", "peak_source": f"copy bandwidth ({src} peaks)"}
+    roof["frac"] = roof["achieved"] / peak if peak else None
+    return {"what": what, "ms_per_launch": ms, "replays": reps, "window_ms": window, "roofline": roof,
+            "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")}, "cpu_baseline": cpu}
+
+
+def measure_next_rows(dg, torch, args, dev, local) -> dict:
+    """The rows beyond the GEMM of the headline path, each timed like the
+    workloads (CUDA-graph replays, median per launch), against its roofline,
+    with the oracle's rate on a bounded sample (--next-cpu-seconds each):
+    activation quantisation, the MoE permutation and combine around the
+    contiguous GEMM, the NN / TN / TT operand layouts, FP32 output plus C, and
+    the 1D1D recipe (both on the dense 4096 x 7168 x 2048 problem)."""
+    from oracle import fp8_gemm as oracle
+    from moe_grouped_gemm_05_b200 import synth
+
+    secs = 0 if args.no_cpu_baseline else args.next_cpu_seconds
+    rows = {}
+    gen = torch.Generator(device=dev)
+    f8 = torch.float8_e4m3fn
+
+    # activation quantisation: the contiguous workload's 32768 x 7168 BF16 activations
+    M, K = 32768, NEXT_K
+    gen.manual_seed(2001)
+    x = torch.randn((M, K), generator=gen, device=dev).to(torch.bfloat16)
+    q = torch.empty((M, K), dtype=f8, device=dev)
+    sf = torch.empty(dg.packed_sf_words(M, K // 128), dtype=torch.int32, device=dev)
+    kp, mn4 = dg.packed_sf_words(M, K // 128)
+    t = _graph_time(lambda i: dg.quantize_fp8_1x128(x, q=q, sf=sf), torch, args, local)
+    cpu = None
+    if secs:
+        xs = x[:4096].float().cpu().numpy()
+        cpu = _timed_cpu(lambda n: oracle.quantize_fp8_1x128(xs[:n]), secs,
+                         lambda n, s: (n * K * 3 / s / 1e9, "GB/s"),
+                         lambda n: 4096 if n is None else f"first {n} of the {M} rows x K={K}")
+    rows["quantize_fp8_1x128"] = _next_row(f"BF16 [{M}, {K}] -> E4M3 + packed UE8M0 (1x128)", t,
+                                           nbytes=M * K * 2 + M * K + 4 * kp * mn4, cpu=cpu)
+    del x, q, sf
+
+    # MoE permutation (routing + gather into the contiguous layout) and the weighted combine
+    T, topk, G, N = NEXT_T, NEXT_TOPK, NEXT_G, NEXT_N
+    ids, gates = synth.topk_routing(2002, T, topk, G)
+    ids_d, gates_d = torch.from_numpy(ids).to(dev), torch.from_numpy(gates).to(dev)
+    gen.manual_seed(2003)
+    qt, sft = dg.quantize_fp8_1x128(torch.randn((T, K), generator=gen, device=dev).to(torch.bfloat16))
+    per = dg.moe_permute(ids_d, G, qt, sft)
+    cap = per["a"].shape[0]
+    routed = T * topk
+    kp_t = (K // 128 + 3) // 4
+    t = _graph_time(lambda i: dg.moe_permute(ids_d, G, qt, sft, out=per), torch, args, local)
+    cpu = None
+    if secs:
+        qh = qt.view(torch.uint8).cpu().numpy()
+
+        def permute_cpu(n):
+            m_idx, row_of, src_of, total, bad = oracle.moe_permute(ids[:n], G)
+            return qh[src_of[src_of >= 0]]
+
+        cpu = _timed_cpu(permute_cpu, secs, lambda n, s: (n * topk * K * 2 / s / 1e9, "GB/s"),
+                         lambda n: T if n is None else f"first {n} of the {T} tokens (top-{topk} of {G})")
+    rows["moe_permute"] = _next_row(
+        f"{T} tokens top-{topk} over {G} experts -> contiguous layout ({cap} rows), K={K}", t,
+        nbytes=T * K + 4 * T * kp_t + 4 * routed + routed * K + 4 * routed * kp_t + 8 * cap + 4 * routed, cpu=cpu)
+    gen.manual_seed(2004)
+    dperm = torch.randn((cap, N), generator=gen, device=dev).to(torch.bfloat16)
+    out = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+    t = _graph_time(lambda i: dg.moe_unpermute_combine(dperm, per["row_of"], gates_d, out=out), torch, args, local)
+    cpu = None
+    if secs:
+        row_of = per["row_of"].cpu().numpy()
+        d_bits = dperm[:, :].view(torch.int16).cpu().numpy().view(np.uint16)
+
+        def combine_cpu(n):
+            r = row_of[:n].reshape(-1)
+            return oracle.moe_unpermute_combine(d_bits[r], np.arange(len(r), dtype=np.int32).reshape(n, topk),
+                                                gates[:n])
+
+        cpu = _timed_cpu(combine_cpu, secs, lambda n, s: ((n * topk * N * 2 + n * N * 2) / s / 1e9, "GB/s"),
+                         lambda n: T if n is None else f"first {n} of the {T} tokens x N={N}")
+    rows["moe_unpermute_combine"] = _next_row(f"{T} tokens x top-{topk} BF16 rows of N={N} -> weighted sum", t,
+                                              nbytes=routed * N * 2 + 8 * routed + T * N * 2, cpu=cpu)
+    del qt, sft, per, dperm, out
+
+    # the dense 4096 x 7168 x 2048 problem in the other operand layouts, FP32 output + C, and 1D1D
+    p = synth.WORKLOADS["dense_4096x7168x2048"]()
+    M, N, K = p.M, p.N, p.K
+    flops = p.flops
+    sfa = dg.pack_sf_ue8m0(torch.from_numpy(np.ascontiguousarray(p.sfa)).to(dev))
+    sfb = dg.pack_sf_ue8m0(torch.from_numpy(np.ascontiguousarray(p.sfb)).to(dev))
+    nsets = 4  # 4 x (A + B + D) = 330 MB > 2x L2
+    to = lambda arr: torch.from_numpy(np.ascontiguousarray(arr)).to(dev).view(f8)  # noqa: E731
+    gemm_cpu = None
+    if secs:
+        smp = OracleSample(p)
+        r = smp.calibrate(secs)
+        gemm_cpu = smp.info(r, smp.run(r))
+    for layout in ("nn", "tn", "tt"):
+        a_s = to(p.a.T) if layout[0] == "t" else to(p.a)
+        b_s = to(p.b.T) if layout[1] == "n" else to(p.b)
+        sets = [(a_s if i == 0 else a_s.clone(), b_s if i == 0 else b_s.clone(),
+                 torch.empty((M, N), dtype=torch.bfloat16, device=dev)) for i in range(nsets)]
+        t = _graph_time(lambda i: dg.fp8_gemm(layout, sets[i % nsets][0], sfa, sets[i % nsets][1], sfb,
+                                              sets[i % nsets][2]), torch, args, local)
+        rows[f"fp8_gemm_{layout}"] = _next_row(
+            f"dense {M}x{N}x{K}, A stored {'[K][M]' if layout[0] == 't' else '[M][K]'}, "
+            f"B stored {'[K][N]' if layout[1] == 'n' else '[N][K]'}", t, flops=flops,
+            nbytes=M * K + N * K + 2 * M * N, cpu=gemm_cpu)
+        del sets, a_s, b_s
+    a, b = to(p.a), to(p.b)
+    gen.manual_seed(2005)
+    c = torch.randn((M, N), generator=gen, device=dev)
+    dsets = [torch.empty((M, N), dtype=torch.float32, device=dev) for _ in range(2)]
+    t = _graph_time(lambda i: dg.fp8_gemm_nt_ex(a, sfa, b, sfb, c=c, d=dsets[i % 2], out_dtype=torch.float32),
+                    torch, args, local)
+    cpu = None
+    if secs:
+        sa_w, sb_w = oracle.pack_sf_ue8m0(p.sfa[None])[0][0], oracle.pack_sf_ue8m0(p.sfb[None])[0][0]
+        ch = c[:1024].cpu().numpy()
+        cpu = _timed_cpu(lambda n: oracle.fp8_gemm_nt_general_f64(p.a, sa_w, p.b, sb_w, M, N, K, c=ch,
+                                                                  rows=np.arange(n)), secs,
+                         lambda n, s: (2.0 * n * N * K / s / 1e12, "TFLOPS"),
+                         lambda n: 1024 if n is None else f"first {n} rows x all {N} columns x K={K}")
+    rows["fp8_gemm_nt_ex_fp32_plus_c"] = _next_row(f"dense {M}x{N}x{K}, FP32 D = A.B^T + C (FP32 C)", t, flops=flops,
+                                                   nbytes=M * K + N * K + 8 * M * N, cpu=cpu)
+    del c, dsets
+    # 1D1D: one scale per row of B (each 128x128 block's scale repeated over its rows)
+    sfb_rows = np.ascontiguousarray(np.repeat(p.sfb, 128, axis=0)[:N])
+    sfb1 = dg.pack_sf_ue8m0(torch.from_numpy(sfb_rows).to(dev))
+    dsets = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    asets = [a if i == 0 else a.clone() for i in range(nsets)]
+    t = _graph_time(lambda i: dg.fp8_gemm_nt_ex(asets[i % nsets], sfa, b, sfb1, d=dsets[i % nsets], recipe_b=1),
+                    torch, args, local)
+    cpu = None
+    if secs:
+        sa_w = oracle.pack_sf_ue8m0(p.sfa[None])[0][0]
+        sb1_w = oracle.pack_sf_ue8m0(sfb_rows[None])[0][0]
+        cpu = _timed_cpu(lambda n: oracle.fp8_gemm_nt_general_f64(p.a, sa_w, p.b, sb1_w, M, N, K, sfb_gran_n=1,
+                                                                  rows=np.arange(n)), secs,
+                         lambda n, s: (2.0 * n * N * K / s / 1e12, "TFLOPS"),
+                         lambda n: 1024 if n is None else f"first {n} rows x all {N} columns x K={K}")
+    rows["fp8_gemm_nt_ex_1d1d"] = _next_row(f"dense {M}x{N}x{K}, B with one scale per row and 128-K block", t,
+                                            flops=flops, nbytes=M * K + N * K + 2 * M * N, cpu=cpu)
+    del asets, dsets, a, b
+    torch.cuda.synchronize()
+    assert dg.get_device_error() == 0, "device error word set during the next-row measurements"
+    torch.cuda.empty_cache()
+    return rows
+
+
 def e2e_loop(p, m, dg, lib, torch, args, barrier):
     """End to end through the public API: every step copies its inputs from
     pinned host memory, packs + multiplies, and copies D back to pinned host
@@ -759,6 +996,9 @@ def run_ours(args):
         line["workloads"][name] = entry
     if rank == 0 and world == 1 and not args.no_cpu_baseline and "cpu_baseline" not in line:
         line["cpu_baseline"] = cpu_baseline_of(full, args.cpu_seconds)
+    # the rows beyond the headline's GEMM (one GPU, full runs only)
+    if world == 1 and args.workloads != "none" and not args.no_next_rows and not args.eager:
+        line["next_rows"] = measure_next_rows(dg, torch, args, dev, local)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

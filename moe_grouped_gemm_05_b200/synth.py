@@ -146,6 +146,20 @@ def zipf_counts(seed: int, rows: int, groups: int, s: float) -> np.ndarray:
     return np.bincount(e, minlength=groups).astype(np.int64)
 
 
+def topk_routing(seed: int, tokens: int, topk: int, groups: int, s: float = 1.1):
+    """Top-k routing of ``tokens`` tokens over ``groups`` experts: each token's
+    ``topk`` distinct experts drawn without replacement with Zipf(s) weights
+    over ranks 1..groups (the largest of log w_e + Gumbel noise, the noise
+    from SplitMix64 uniforms), and gate weights that sum to one per token.
+    Returns (ids int32 [tokens, topk], gates float32 [tokens, topk])."""
+    w = np.arange(1, groups + 1, dtype=np.float64) ** (-s)
+    u = np.clip(uniform01(seed, 0, tokens * groups), 1e-300, None).reshape(tokens, groups)
+    keys = np.log(w)[None, :] - np.log(-np.log(u))
+    ids = np.argsort(-keys, axis=1, kind="stable")[:, :topk].astype(np.int32)
+    g = uniform01(seed ^ 0x5151, 0, tokens * topk).reshape(tokens, topk) + 0.5
+    return ids, (g / g.sum(axis=1, keepdims=True)).astype(np.float32)
+
+
 def contiguous_indices(counts: np.ndarray, align: int = BLOCK) -> np.ndarray:
     """Per-row expert index for segments of ``counts`` rows, each padded with -1 to ``align``."""
     parts = []

@@ -352,6 +352,22 @@ def test_zipf_routing_counts():
     assert len(idx) % 128 == 0 and (idx >= 0).sum() == 32768
 
 
+def test_topk_routing():
+    """Top-1 routing by largest log-weight + Gumbel noise is a Zipf draw; top-k
+    slots of a token are distinct experts; gates sum to one; the draw is seeded."""
+    ids, g = synth.topk_routing(5, 40000, 1, 8, 1.1)
+    c = np.bincount(ids[:, 0], minlength=8)
+    p = np.arange(1, 9) ** -1.1
+    expect = 40000 * p / p.sum()
+    assert np.all(np.abs(c - expect) < 5 * np.sqrt(expect))
+    ids2, g2 = synth.topk_routing(6, 5000, 3, 8, 1.1)
+    assert ids2.shape == (5000, 3) and ids2.min() >= 0 and ids2.max() < 8
+    assert all(len(set(r)) == 3 for r in ids2.tolist())
+    assert np.allclose(g2.sum(axis=1), 1.0) and (g2 > 0).all()
+    again, _ = synth.topk_routing(6, 5000, 3, 8, 1.1)
+    assert np.array_equal(ids2, again)
+
+
 def test_masked_counts_range():
     m = synth.uniform_masked_m(7, 1000, 256)
     assert m.min() >= 0 and m.max() <= 256 and 100 < m.mean() < 156
