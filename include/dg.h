@@ -209,6 +209,7 @@ int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int 
  * feed dg_m_grouped_fp8_gemm_nt_contiguous with M_total = M_cap directly.
  * Ids outside [-1, num_experts) set DG_DEVERR_BAD_EXPERT and are not routed.
  * num_experts <= 1024; M_cap >= dg_moe_permute_capacity(...) and a multiple of 128.
+ * With T = 0, topk_ids, q, sfa and row_of may be NULL: every row becomes padding.
  * dg_moe_unpermute_combine:
  *   out[t] = bf16_rne( sum_s weights[t][s] * d_perm[row_of[t][s]] ) in FP32 over routed
  *   slots (weights NULL = 1); d_perm BF16 [rows][N], out BF16 [T][N], N % 16 == 0.

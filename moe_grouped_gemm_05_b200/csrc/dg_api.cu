@@ -105,19 +105,24 @@ struct LaunchAttrs {
   }
 };
 
-// cudaLaunchKernelEx of a plain (non-cluster) kernel with the PDL attribute.
+// cudaLaunchKernelEx of a kernel with the PDL attribute (and clusters of `cluster` CTAs).
 template <typename... Params, typename... Args>
-static cudaError_t launch_plain(void (*kernel)(Params...), long long blocks, int threads, cudaStream_t st,
-                                Args&&... args) {
-  LaunchAttrs la(1);
+static cudaError_t launch_plain_smem(void (*kernel)(Params...), long long blocks, int threads, size_t smem,
+                                     cudaStream_t st, int cluster, Args&&... args) {
+  LaunchAttrs la(cluster);
   cudaLaunchConfig_t lc = {};
   lc.gridDim = dim3(static_cast<unsigned>(blocks));
   lc.blockDim = dim3(threads);
-  lc.dynamicSmemBytes = 0;
+  lc.dynamicSmemBytes = smem;
   lc.stream = st;
   lc.attrs = la.attr;
   lc.numAttrs = la.n;
   return cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+}
+template <typename... Params, typename... Args>
+static cudaError_t launch_plain(void (*kernel)(Params...), long long blocks, int threads, cudaStream_t st,
+                                Args&&... args) {
+  return launch_plain_smem(kernel, blocks, threads, 0, st, 1, std::forward<Args>(args)...);
 }
 static thread_local int t_force_bn = 0;
 
@@ -837,8 +842,8 @@ int dg_moe_permute_capacity(int T, int topk, int num_experts) {
 int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, const void* q, const int32_t* sfa, int K,
                    void* a_perm, int32_t* sfa_perm, int32_t* m_indices, int32_t* row_of, int32_t* src_of, int M_cap,
                    void* stream) {
-  if (!topk_ids || !q || !sfa || !a_perm || !sfa_perm || !m_indices || !row_of || !src_of)
-    return fail(DG_ERR_NULL, "every pointer must be non-NULL");
+  if (!a_perm || !sfa_perm || !m_indices || !src_of || (T != 0 && (!topk_ids || !q || !sfa || !row_of)))
+    return fail(DG_ERR_NULL, "every pointer must be non-NULL (topk_ids, q, sfa and row_of may be NULL when T = 0)");
   if (!aligned16(q) || !aligned16(a_perm) || !aligned16(sfa) || !aligned16(sfa_perm))
     return fail(DG_ERR_ALIGN, "q, sfa, a_perm and sfa_perm must be 16-byte aligned");
   if (T < 0 || topk <= 0 || num_experts <= 0 || num_experts > kMoeMaxExperts)
@@ -854,13 +859,37 @@ int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, co
   int r = device_info(&di);
   if (r) return r;
   auto st = static_cast<cudaStream_t>(stream);
-  DG_CUDA_TRY(launch_plain(moe_route_kernel, num_experts, kMoeThreads, st, topk_ids, static_cast<int>(n), topk,
-                           num_experts, M_cap, m_indices, row_of, src_of));
   const int kp = (K / 128 + 3) / 4;
-  const long long work = static_cast<long long>(M_cap) * (K / 16);
+  // one CTA per expert, in whole clusters
+  const int route_ctas = (num_experts + kRouteCluster - 1) / kRouteCluster * kRouteCluster;
+  if (n <= kMoeStagedIds) {
+    // every routing id fits in shared memory: each CTA reads them from global memory once
+    static std::mutex mu;
+    static bool attr_done[64] = {};
+    int dev = 0;
+    DG_CUDA_TRY(cudaGetDevice(&dev));
+    {
+      std::lock_guard<std::mutex> lock(mu);
+      if (dev < 0 || dev >= 64) return fail(DG_ERR_UNSUPPORTED, "device %d outside the launch table", dev);
+      if (!attr_done[dev]) {
+        DG_CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(&moe_route_kernel<true>),
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMoeStagedIds * 4));
+        attr_done[dev] = true;
+      }
+    }
+    DG_CUDA_TRY(launch_plain_smem(moe_route_kernel<true>, route_ctas, kMoeThreads, static_cast<size_t>(n) * 4, st,
+                                  kRouteCluster, topk_ids, static_cast<int>(n), topk, num_experts, M_cap, kp,
+                                  m_indices, row_of, src_of, reinterpret_cast<uint32_t*>(sfa_perm)));
+  } else {
+    DG_CUDA_TRY(launch_plain_smem(moe_route_kernel<false>, route_ctas, kMoeThreads, 0, st, kRouteCluster, topk_ids,
+                                  static_cast<int>(n), topk, num_experts, M_cap, kp, m_indices, row_of, src_of,
+                                  reinterpret_cast<uint32_t*>(sfa_perm)));
+  }
+  const long long work = static_cast<long long>(T) * (K / 16);
+  if (work == 0) return DG_OK;
   const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 16LL * di.sms));
   DG_CUDA_TRY(launch_plain(moe_gather_kernel, blocks, 256, st, static_cast<const uint8_t*>(q),
-                           reinterpret_cast<const uint32_t*>(sfa), T, K, kp, static_cast<const int32_t*>(src_of),
+                           reinterpret_cast<const uint32_t*>(sfa), T, K, kp, topk, static_cast<const int32_t*>(row_of),
                            M_cap, static_cast<uint8_t*>(a_perm), reinterpret_cast<uint32_t*>(sfa_perm)));
   return DG_OK;
 }

@@ -3,14 +3,17 @@
 // group_by_expert step before the grouped GEMM and the combine after it;
 // juejin.cn §4 "分组 GEMM（连续布局）": expert segments aligned to the M block).
 //
-// moe_route_kernel   one CTA per expert: histogram of all routing ids in
-//                    shared memory -> this expert's segment offset (segments
-//                    in expert order, each padded to 128 rows) -> a stable
-//                    compaction of the (token, slot) pairs routed to it
-//                    (warp ballots + a block scan), so the layout is
-//                    deterministic.  Writes m_indices, src_of and row_of.
-// moe_gather_kernel  full grid: copies each routed row's FP8 codes and its
-//                    packed scale words to its destination row.
+// moe_route_kernel   one CTA per expert, in clusters: the cluster's CTAs
+//                    split the histogram of all routing ids and add it up
+//                    through distributed shared memory -> each expert's
+//                    segment offset (segments in expert order, each padded to
+//                    128 rows) -> a stable compaction of the (token, slot)
+//                    pairs routed to the CTA's expert (a block scan), so the
+//                    layout is deterministic.  Writes m_indices, src_of,
+//                    row_of, and zero scale words for padding rows.
+// moe_gather_kernel  full grid, tokens in source order: copies each token's
+//                    FP8 codes and packed scale words to the rows of its
+//                    routed slots (one read of each token row).
 // moe_combine_kernel out[t] = bf16(sum_s w[t,s] * D[row_of[t,s]]), FP32 sums.
 #pragma once
 #include <cuda_bf16.h>
@@ -22,106 +25,194 @@ namespace dg {
 
 constexpr int kMoeMaxExperts = 1024;
 constexpr int kMoeThreads = 1024;
+// Routed slots up to which the routing kernel stages all ids in shared memory (192 KB).
+constexpr int kMoeStagedIds = 48 * 1024;
 
+// CTAs per cluster of the routing kernel: the cluster's CTAs split the
+// histogram of the ids and add their slices through distributed shared memory.
+constexpr int kRouteCluster = 8;
+
+// One CTA per expert (the grid is G rounded up to whole clusters).
+// kStaged: every CTA first copies the n ids into dynamic shared memory
+// (n <= kMoeStagedIds), so it reads them from global memory once.
+// 1. CTA r of a cluster counts the ids of slice r (1/kRouteCluster of them)
+//    for every expert, and marks that slice's unrouted slots;
+// 2. the cluster adds the slice counts through distributed shared memory,
+//    and every CTA derives the segment offsets (expert order, 128-aligned);
+// 3. CTA e compacts the slots routed to expert e, in slot order (16 slots a
+//    thread per chunk, a block scan orders the threads), and pads its segment.
+template <bool kStaged>
 __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int topk,
-                                                                int G, int M_cap, int32_t* __restrict__ m_indices,
+                                                                int G, int M_cap, int kp, int32_t* __restrict__ m_indices,
                                                                 int32_t* __restrict__ row_of,
-                                                                int32_t* __restrict__ src_of) {
-  __shared__ int cnt[kMoeMaxExperts];
-  __shared__ int warp_tot[32];
-  __shared__ int seg_off, total_rows, running;
+                                                                int32_t* __restrict__ src_of,
+                                                                uint32_t* __restrict__ sfa_perm) {
+  __shared__ int cnt[kMoeMaxExperts];  // this CTA's slice counts
+  __shared__ int tot[kMoeMaxExperts];  // the whole histogram
+  __shared__ int warp_tot[2][32];      // double-buffered by chunk parity: one barrier pair per chunk
+  __shared__ int chunk_off[2];
+  __shared__ int seg_off, total_rows;
+  extern __shared__ __align__(16) int32_t ids_s[];  // kStaged: ids[0, n)
   grid_dep_wait();
   grid_dep_launch();
   const int e = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = blockDim.x >> 5;
+  const int crank = static_cast<int>(cluster_cta_rank());
   for (int i = tid; i < G; i += blockDim.x) cnt[i] = 0;
-  __syncthreads();
-  for (int i = tid; i < n; i += blockDim.x) {
-    const int v = __ldg(&ids[i]);
-    if (v >= 0 && v < G) atomicAdd(&cnt[v], 1);
-    else if (v != -1 && e == 0) atomicOr(&g_dg_error, 0x2);
+  if constexpr (kStaged) {
+    // 8 independent loads in flight per thread, then their stores
+    for (int base = 0; base < n; base += 8 * kMoeThreads) {
+      int r[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kMoeThreads + tid;
+        r[j] = i < n ? __ldg(&ids[i]) : 0;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = base + j * kMoeThreads + tid;
+        if (i < n) ids_s[i] = r[j];
+      }
+    }
   }
+  auto id_at = [&](int i) -> int {
+    if constexpr (kStaged) return ids_s[i];
+    else return __ldg(&ids[i]);
+  };
   __syncthreads();
+  // 1. this CTA's slice: counts (lanes holding the same id add once per warp),
+  //    unrouted and out-of-range slots
+  const int slice = (n + kRouteCluster - 1) / kRouteCluster;
+  const int s0 = min(n, crank * slice), s1 = min(n, s0 + slice);
+  for (int base = s0; base < s1; base += blockDim.x) {
+    const int i = base + tid;
+    const int v = i < s1 ? id_at(i) : -1;
+    if (i < s1 && (v < 0 || v >= G)) row_of[i] = -1;
+    if (__any_sync(0xffffffffu, i < s1 && !(v >= -1 && v < G)) && lane == 0) atomicOr(&g_dg_error, 0x2);
+    const unsigned same = __match_any_sync(0xffffffffu, v);
+    if (v >= 0 && v < G && lane == __ffs(same) - 1) atomicAdd(&cnt[v], __popc(same));
+  }
+  cluster_sync();
+  // 2. the histogram: the sum of the cluster's slice counts
+  for (int g = tid; g < G; g += blockDim.x) {
+    const uint32_t a = smem_u32(&cnt[g]);
+    int t = 0;
+#pragma unroll
+    for (int c = 0; c < kRouteCluster; ++c) t += static_cast<int>(ld_shared_cluster_u32(mapa_shared(a, c)));
+    tot[g] = t;
+  }
+  cluster_sync();  // every CTA has read every slice: from here none reads a peer
   if (tid == 0) {
-    int off = 0, tot = 0;
+    int off = 0, all = 0;
     for (int g = 0; g < G; ++g) {
-      const int padded = (cnt[g] + 127) & ~127;
+      const int padded = (tot[g] + 127) & ~127;
       if (g < e) off += padded;
-      tot += padded;
+      all += padded;
     }
     seg_off = off;
-    total_rows = tot;
-    running = 0;
+    total_rows = all;
+    chunk_off[0] = 0;
   }
   __syncthreads();
-  // stable compaction of the slots routed to expert e
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + tid;
-    const bool flag = i < n && __ldg(&ids[i]) == e;
-    const unsigned ballot = __ballot_sync(0xffffffffu, flag);
-    if (lane == 0) warp_tot[warp] = __popc(ballot);
+  if (e >= G) return;  // a CTA that only completes the last cluster
+  // 3. stable compaction of the slots routed to expert e
+  int par = 0;
+  for (int base = 0; base < n; base += 16 * kMoeThreads, par ^= 1) {
+    const int i0 = base + 16 * tid;
+    unsigned flags = 0;
+    if (kStaged && i0 + 15 < n) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int4 v4 = reinterpret_cast<const int4*>(ids_s + i0)[q];  // i0 is a multiple of 16: aligned
+        flags |= (static_cast<unsigned>(v4.x == e) | (static_cast<unsigned>(v4.y == e) << 1) |
+                  (static_cast<unsigned>(v4.z == e) << 2) | (static_cast<unsigned>(v4.w == e) << 3))
+                 << (4 * q);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int i = i0 + j;
+        flags |= static_cast<unsigned>(i < n && id_at(i) == e) << j;
+      }
+    }
+    const int c = __popc(flags);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += u;
+    }
+    if (lane == 31) warp_tot[par][warp] = incl;
     __syncthreads();
     if (warp == 0) {
-      const int nw = blockDim.x >> 5;
-      int v = lane < nw ? warp_tot[lane] : 0;
-      int incl = v;
+      const int v = lane < nw ? warp_tot[par][lane] : 0;
+      int x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += u;
+        const int u = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += u;
       }
-      if (lane < nw) warp_tot[lane] = incl - v;  // exclusive
+      if (lane < nw) warp_tot[par][lane] = x - v;  // exclusive prefix of the warps
+      if (lane == 31) chunk_off[par ^ 1] = chunk_off[par] + x;
     }
     __syncthreads();
-    if (flag) {
-      const int pos = seg_off + running + warp_tot[warp] + __popc(ballot & ((1u << lane) - 1u));
+    int pos = seg_off + chunk_off[par] + warp_tot[par][warp] + incl - c;
+    while (flags != 0u) {
+      const int i = i0 + __ffs(flags) - 1;
+      flags &= flags - 1u;
       m_indices[pos] = e;
       src_of[pos] = i / topk;
       row_of[i] = pos;
+      ++pos;
     }
-    __syncthreads();
-    if (tid == blockDim.x - 1) running += warp_tot[warp] + __popc(ballot);
-    __syncthreads();
   }
-  // padding rows of this segment; CTA 0 also marks the tail and the unrouted slots
-  const int c = cnt[e];
-  const int padded = (c + 127) & ~127;
-  for (int r = seg_off + c + tid; r < seg_off + padded; r += blockDim.x) {
+  // padding rows of this segment (scale words 0); CTA 0 also marks the tail past the last segment
+  const int c = tot[e];
+  const int pad0 = seg_off + c, pad1 = seg_off + ((c + 127) & ~127);
+  for (int r = pad0 + tid; r < pad1; r += blockDim.x) {
     m_indices[r] = -1;
     src_of[r] = -1;
   }
+  for (int u = tid; u < (pad1 - pad0) * kp; u += blockDim.x)
+    sfa_perm[static_cast<size_t>(u / (pad1 - pad0)) * M_cap + pad0 + u % (pad1 - pad0)] = 0u;
   if (e == 0) {
     for (int r = total_rows + tid; r < M_cap; r += blockDim.x) {
       m_indices[r] = -1;
       src_of[r] = -1;
     }
-    for (int i = tid; i < n; i += blockDim.x) {
-      const int v = __ldg(&ids[i]);
-      if (v < 0 || v >= G) row_of[i] = -1;
-    }
+    const int tail = M_cap - total_rows;
+    for (long long u = tid; u < static_cast<long long>(tail) * kp; u += blockDim.x)
+      sfa_perm[static_cast<size_t>(u / tail) * M_cap + total_rows + u % tail] = 0u;
   }
 }
 
-// a_perm[r] = q[src_of[r]] (K bytes) and sfa_perm[kp][r] = sfa[kp][src_of[r]];
-// padding rows get scale words 0 and keep whatever codes they held.
+// a_perm[row_of[t][s]] = q[t] (K bytes) and sfa_perm[kp][row_of[t][s]] =
+// sfa[kp][t] for every routed slot s of token t: tokens in source order, so
+// each token's row is read once however many slots it has.  Padding and tail
+// rows keep whatever codes they held (their scale words are zeroed by
+// moe_route_kernel).
 __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restrict__ q, const uint32_t* __restrict__ sfa,
-                                                        int T, int K, int kp, const int32_t* __restrict__ src_of,
-                                                        int M_cap, uint8_t* __restrict__ a_perm,
-                                                        uint32_t* __restrict__ sfa_perm) {
+                                                        int T, int K, int kp, int topk,
+                                                        const int32_t* __restrict__ row_of, int M_cap,
+                                                        uint8_t* __restrict__ a_perm, uint32_t* __restrict__ sfa_perm) {
   grid_dep_wait();
   grid_dep_launch();
   const int chunks = K / 16;
   const int t4 = (T + 3) & ~3;
-  const long long total = static_cast<long long>(M_cap) * chunks;
+  const long long total = static_cast<long long>(T) * chunks;
   for (long long u = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u < total;
        u += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int r = static_cast<int>(u / chunks);
-    const int ch = static_cast<int>(u - static_cast<long long>(r) * chunks);
-    const int t = __ldg(&src_of[r]);
-    if (t >= 0)
-      reinterpret_cast<uint4*>(a_perm + static_cast<size_t>(r) * K)[ch] =
-          __ldg(reinterpret_cast<const uint4*>(q + static_cast<size_t>(t) * K) + ch);
-    if (ch < kp) sfa_perm[static_cast<size_t>(ch) * M_cap + r] = t >= 0 ? __ldg(&sfa[static_cast<size_t>(ch) * t4 + t]) : 0u;
+    const int t = static_cast<int>(u / chunks);
+    const int ch = static_cast<int>(u - static_cast<long long>(t) * chunks);
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + static_cast<size_t>(t) * K) + ch);
+    const uint32_t w = ch < kp ? __ldg(&sfa[static_cast<size_t>(ch) * t4 + t]) : 0u;
+    for (int s = 0; s < topk; ++s) {
+      const int r = __ldg(&row_of[static_cast<size_t>(t) * topk + s]);
+      if (r < 0) continue;
+      reinterpret_cast<uint4*>(a_perm + static_cast<size_t>(r) * K)[ch] = v;
+      if (ch < kp) sfa_perm[static_cast<size_t>(ch) * M_cap + r] = w;
+    }
   }
 }
 

@@ -54,6 +54,57 @@ def test_permute_bit_exact(T, topk, G, K):
     assert (sf_out[:, gm < 0] == 0).all()
 
 
+def test_permute_into_prefilled_buffers_over_many_chunks():
+    """15000 routed slots (several 4096-slot compaction chunks and a ragged
+    last one) with Zipf-weighted top-3 routing, into output buffers filled with
+    garbage first: every index, row and scale word the contract defines is
+    written, padding and tail scale words included."""
+    T, topk, G, K = 5000, 3, 8, 384
+    ids, _ = synth.topk_routing(41, T, topk, G)
+    ids[::7, 1] = -1  # some unrouted slots
+    x = torch.from_numpy(synth.normal(42, T * K).reshape(T, K)).to(torch.bfloat16).cuda()
+    q, sfa = dg.quantize_fp8_1x128(x)
+    cap = dg.load().dg_moe_permute_capacity(T, topk, G)
+    kp = (K // 128 + 3) // 4
+    out = {"a": torch.full((cap, K), 0x7E, dtype=torch.uint8, device="cuda").view(torch.float8_e4m3fn),
+           "sfa": torch.full((kp, cap), 0x5A5A5A5A, dtype=torch.int32, device="cuda"),
+           "m_indices": torch.full((cap,), 77, dtype=torch.int32, device="cuda"),
+           "src_of": torch.full((cap,), 77, dtype=torch.int32, device="cuda"),
+           "row_of": torch.full((T, topk), 77, dtype=torch.int32, device="cuda")}
+    dg.moe_permute(torch.from_numpy(ids).cuda(), G, q, sfa, out=out)
+    torch.cuda.synchronize()
+    assert dg.get_device_error() == 0
+    m, row_of, src, Mt, bad = oracle.fp8_gemm.moe_permute(ids, G)
+    gm, gs = out["m_indices"].cpu().numpy(), out["src_of"].cpu().numpy()
+    assert np.array_equal(gm[:Mt], m) and (gm[Mt:] == -1).all()
+    assert np.array_equal(gs[:Mt], src) and (gs[Mt:] == -1).all()
+    assert np.array_equal(out["row_of"].cpu().numpy(), row_of)
+    valid = np.nonzero(m >= 0)[0]
+    an = out["a"].view(torch.uint8).cpu().numpy()
+    assert np.array_equal(an[valid], q.view(torch.uint8).cpu().numpy()[src[valid]])
+    sf_out = out["sfa"].cpu().numpy()
+    assert np.array_equal(sf_out[:, valid], sfa.cpu().numpy()[:, src[valid]])
+    assert (sf_out[:, gm < 0] == 0).all()
+
+
+def test_permute_no_tokens_marks_every_row_padding():
+    K, G, topk = 256, 4, 2
+    cap = dg.load().dg_moe_permute_capacity(0, topk, G)
+    kp = (K // 128 + 3) // 4
+    out = {"a": torch.zeros((cap, K), dtype=torch.float8_e4m3fn, device="cuda"),
+           "sfa": torch.full((kp, cap), 9, dtype=torch.int32, device="cuda"),
+           "m_indices": torch.full((cap,), 9, dtype=torch.int32, device="cuda"),
+           "src_of": torch.full((cap,), 9, dtype=torch.int32, device="cuda"),
+           "row_of": torch.zeros((0, topk), dtype=torch.int32, device="cuda")}
+    q = torch.zeros((0, K), dtype=torch.float8_e4m3fn, device="cuda")
+    sfa = torch.zeros(dg.packed_sf_words(0, K // 128), dtype=torch.int32, device="cuda")
+    dg.moe_permute(torch.zeros((0, topk), dtype=torch.int32, device="cuda"), G, q, sfa, out=out)
+    torch.cuda.synchronize()
+    assert (out["m_indices"].cpu().numpy() == -1).all() and (out["src_of"].cpu().numpy() == -1).all()
+    assert (out["sfa"].cpu().numpy() == 0).all()
+    assert dg.get_device_error() == 0
+
+
 def test_permute_flags_bad_ids():
     ids = np.array([[0, 5], [1, -3]], np.int32)
     x = torch.ones((2, 128), dtype=torch.bfloat16, device="cuda")
