@@ -860,34 +860,28 @@ int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, co
   if (r) return r;
   auto st = static_cast<cudaStream_t>(stream);
   const int kp = (K / 128 + 3) / 4;
-  // one CTA per expert, in whole clusters
-  const int route_ctas = (num_experts + kRouteCluster - 1) / kRouteCluster * kRouteCluster;
-  if (n <= kMoeStagedIds) {
-    // every routing id fits in shared memory: each CTA reads them from global memory once
+  // the routing kernel: one cluster; its table needs more than 48 KB of shared memory beyond 320 experts
+  {
     static std::mutex mu;
     static bool attr_done[64] = {};
     int dev = 0;
     DG_CUDA_TRY(cudaGetDevice(&dev));
-    {
-      std::lock_guard<std::mutex> lock(mu);
-      if (dev < 0 || dev >= 64) return fail(DG_ERR_UNSUPPORTED, "device %d outside the launch table", dev);
-      if (!attr_done[dev]) {
-        DG_CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(&moe_route_kernel<true>),
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kMoeStagedIds * 4));
-        attr_done[dev] = true;
-      }
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev < 0 || dev >= 64) return fail(DG_ERR_UNSUPPORTED, "device %d outside the launch table", dev);
+    if (!attr_done[dev]) {
+      DG_CUDA_TRY(cudaFuncSetAttribute(reinterpret_cast<const void*>(&moe_route_kernel),
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, route_smem_bytes(kMoeMaxExperts)));
+      attr_done[dev] = true;
     }
-    DG_CUDA_TRY(launch_plain_smem(moe_route_kernel<true>, route_ctas, kMoeThreads, static_cast<size_t>(n) * 4, st,
-                                  kRouteCluster, topk_ids, static_cast<int>(n), topk, num_experts, M_cap, kp,
-                                  m_indices, row_of, src_of, reinterpret_cast<uint32_t*>(sfa_perm)));
-  } else {
-    DG_CUDA_TRY(launch_plain_smem(moe_route_kernel<false>, route_ctas, kMoeThreads, 0, st, kRouteCluster, topk_ids,
-                                  static_cast<int>(n), topk, num_experts, M_cap, kp, m_indices, row_of, src_of,
-                                  reinterpret_cast<uint32_t*>(sfa_perm)));
   }
+  DG_CUDA_TRY(launch_plain_smem(moe_route_kernel, kRouteCluster, kMoeThreads,
+                                static_cast<size_t>(route_smem_bytes(num_experts)), st, kRouteCluster, topk_ids,
+                                static_cast<int>(n), topk, num_experts, M_cap, kp, m_indices, row_of, src_of,
+                                reinterpret_cast<uint32_t*>(sfa_perm)));
   const long long work = static_cast<long long>(T) * (K / 16);
   if (work == 0) return DG_OK;
-  const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 16LL * di.sms));
+  const long long blocks =
+      std::max<long long>(1, std::min<long long>((work + 256 * kGatherU - 1) / (256 * kGatherU), 8LL * di.sms));
   DG_CUDA_TRY(launch_plain(moe_gather_kernel, blocks, 256, st, static_cast<const uint8_t*>(q),
                            reinterpret_cast<const uint32_t*>(sfa), T, K, kp, topk, static_cast<const int32_t*>(row_of),
                            M_cap, static_cast<uint8_t*>(a_perm), reinterpret_cast<uint32_t*>(sfa_perm)));
@@ -904,10 +898,15 @@ int dg_moe_unpermute_combine(const void* d_perm, const int32_t* row_of, const fl
   DeviceInfo di;
   int r = device_info(&di);
   if (r) return r;
-  const long long blocks = std::min<long long>((work + 255) / 256, 16LL * di.sms);
-  DG_CUDA_TRY(launch_plain(moe_combine_kernel, blocks, 256, static_cast<cudaStream_t>(stream),
-                           static_cast<const __nv_bfloat16*>(d_perm), row_of, weights, T, topk, N,
-                           static_cast<__nv_bfloat16*>(out)));
+  // slots per pass: one at a time up to top-2 (measured fastest there), else 4 or 8 (passes of 8 beyond)
+  const int slots = topk <= 2 ? 1 : topk <= 4 ? 4 : 8;
+  const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 16LL * di.sms));
+  auto st = static_cast<cudaStream_t>(stream);
+  auto dp = static_cast<const __nv_bfloat16*>(d_perm);
+  auto op = static_cast<__nv_bfloat16*>(out);
+  if (slots == 1) DG_CUDA_TRY(launch_plain(moe_combine_kernel<1>, blocks, 256, st, dp, row_of, weights, T, topk, N, op));
+  else if (slots == 4) DG_CUDA_TRY(launch_plain(moe_combine_kernel<4>, blocks, 256, st, dp, row_of, weights, T, topk, N, op));
+  else DG_CUDA_TRY(launch_plain(moe_combine_kernel<8>, blocks, 256, st, dp, row_of, weights, T, topk, N, op));
   return DG_OK;
 }
 

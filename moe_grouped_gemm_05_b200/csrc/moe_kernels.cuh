@@ -3,14 +3,14 @@
 // group_by_expert step before the grouped GEMM and the combine after it;
 // juejin.cn §4 "分组 GEMM（连续布局）": expert segments aligned to the M block).
 //
-// moe_route_kernel   one CTA per expert, in clusters: the cluster's CTAs
-//                    split the histogram of all routing ids and add it up
-//                    through distributed shared memory -> each expert's
-//                    segment offset (segments in expert order, each padded to
-//                    128 rows) -> a stable compaction of the (token, slot)
-//                    pairs routed to the CTA's expert (a block scan), so the
-//                    layout is deterministic.  Writes m_indices, src_of,
-//                    row_of, and zero scale words for padding rows.
+// moe_route_kernel   one cluster of 8 CTAs: a stable counting sort of the
+//                    routed (token, slot) pairs by expert.  Each warp counts
+//                    and later places a run of the slots in slot order; the
+//                    CTAs add their counts through distributed shared memory
+//                    -> each expert's segment offset (segments in expert
+//                    order, each padded to 128 rows), so the layout is
+//                    deterministic.  Writes m_indices, src_of, row_of, and
+//                    zero scale words for padding rows.
 // moe_gather_kernel  full grid, tokens in source order: copies each token's
 //                    FP8 codes and packed scale words to the rows of its
 //                    routed slots (one read of each token row).
@@ -25,173 +25,185 @@ namespace dg {
 
 constexpr int kMoeMaxExperts = 1024;
 constexpr int kMoeThreads = 1024;
-// Routed slots up to which the routing kernel stages all ids in shared memory (192 KB).
-constexpr int kMoeStagedIds = 48 * 1024;
 
-// CTAs per cluster of the routing kernel: the cluster's CTAs split the
-// histogram of the ids and add their slices through distributed shared memory.
+// CTAs of the routing kernel: one cluster, whose CTAs add their counts
+// through distributed shared memory.
 constexpr int kRouteCluster = 8;
+// 32-slot steps of a warp whose ids the routing kernel loads at once.
+constexpr int kRouteSteps = 8;
+// Dynamic shared memory of the routing kernel for G experts: a [32 warps][G]
+// table of counts, then this CTA's slice counts, the expert totals, the
+// earlier CTAs' counts and the segment offsets (G words each).
+__host__ __device__ constexpr int route_smem_bytes(int G) { return (32 * G + 4 * G) * 4; }
 
-// One CTA per expert (the grid is G rounded up to whole clusters).
-// kStaged: every CTA first copies the n ids into dynamic shared memory
-// (n <= kMoeStagedIds), so it reads them from global memory once.
-// 1. CTA r of a cluster counts the ids of slice r (1/kRouteCluster of them)
-//    for every expert, and marks that slice's unrouted slots;
-// 2. the cluster adds the slice counts through distributed shared memory,
-//    and every CTA derives the segment offsets (expert order, 128-aligned);
-// 3. CTA e compacts the slots routed to expert e, in slot order (16 slots a
-//    thread per chunk, a block scan orders the threads), and pads its segment.
-template <bool kStaged>
+// A stable counting sort of the n routed slots by expert, on one cluster of
+// kRouteCluster CTAs of 32 warps.  CTA c owns slots [c*slice, (c+1)*slice),
+// and warp w of it a run of that range in slot order (whole 32-slot steps).
+// 1. every warp counts the slots of its run per expert (match_any: lanes
+//    with the same expert add once, by their first lane), into its row of
+//    the table; unrouted and invalid slots get row_of = -1;
+// 2. the CTA turns the table into exclusive prefixes over its warps and its
+//    slice counts; the cluster adds every CTA's slice counts through
+//    distributed shared memory, giving the expert totals and, per expert,
+//    the slots of the CTAs before this one;
+// 3. a block scan of the 128-padded totals gives the segment offsets (expert
+//    order), and table entry [w][e] becomes the row of warp w's first slot
+//    of expert e;
+// 4. every warp walks its run again in slot order: a slot's row is its
+//    warp's entry plus its rank among the lanes of the step with the same
+//    expert, and the first such lane advances the entry;
+// 5. the padding rows of the segments (experts split over the CTAs) and the
+//    rows past the last segment get index -1 and zero scale words.
 __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int topk,
                                                                 int G, int M_cap, int kp, int32_t* __restrict__ m_indices,
                                                                 int32_t* __restrict__ row_of,
                                                                 int32_t* __restrict__ src_of,
                                                                 uint32_t* __restrict__ sfa_perm) {
-  __shared__ int cnt[kMoeMaxExperts];  // this CTA's slice counts
-  __shared__ int tot[kMoeMaxExperts];  // the whole histogram
-  __shared__ int warp_tot[2][32];      // double-buffered by chunk parity: one barrier pair per chunk
-  __shared__ int chunk_off[2];
-  __shared__ int seg_off, total_rows;
-  extern __shared__ __align__(16) int32_t ids_s[];  // kStaged: ids[0, n)
+  extern __shared__ __align__(16) int rsm[];
+  int* wtab = rsm;             // [32][G]
+  int* ccnt = wtab + 32 * G;   // this CTA's slice counts
+  int* tot = ccnt + G;         // expert totals
+  int* below = tot + G;        // slots of expert e in the CTAs before this one
+  int* seg = below + G;        // segment offsets
+  __shared__ int warp_sum[32];
+  __shared__ int total_rows_s;
   grid_dep_wait();
   grid_dep_launch();
-  const int e = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nw = blockDim.x >> 5;
-  const int crank = static_cast<int>(cluster_cta_rank());
-  for (int i = tid; i < G; i += blockDim.x) cnt[i] = 0;
-  if constexpr (kStaged) {
-    // 8 independent loads in flight per thread, then their stores
-    for (int base = 0; base < n; base += 8 * kMoeThreads) {
-      int r[8];
+  const int c = static_cast<int>(cluster_cta_rank());
+  const int slice = (n + kRouteCluster - 1) / kRouteCluster;
+  const int s0 = min(n, c * slice), s1 = min(n, s0 + slice);
+  const int per_warp = ((s1 - s0 + 32 * 32 - 1) / (32 * 32)) * 32;  // whole 32-slot steps
+  const int w0 = min(s1, s0 + warp * per_warp), w1 = min(s1, w0 + per_warp);
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i = tid; i < 32 * G; i += blockDim.x) wtab[i] = 0;
+  __syncthreads();
+  // 1. per-warp counts (the ids of kRouteSteps steps are loaded at once)
+  int* row = wtab + warp * G;
+  for (int base = w0; base < w1; base += 32 * kRouteSteps) {
+    int vs[kRouteSteps];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + j * kMoeThreads + tid;
-        r[j] = i < n ? __ldg(&ids[i]) : 0;
-      }
+    for (int j = 0; j < kRouteSteps; ++j) {
+      const int i = base + 32 * j + lane;
+      vs[j] = i < w1 ? __ldg(&ids[i]) : -1;
+    }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int i = base + j * kMoeThreads + tid;
-        if (i < n) ids_s[i] = r[j];
-      }
+    for (int j = 0; j < kRouteSteps; ++j) {
+      const int i = base + 32 * j + lane;
+      const int v = vs[j];
+      const bool valid = v >= 0 && v < G;
+      if (i < w1 && !valid) row_of[i] = -1;
+      if (__any_sync(0xffffffffu, i < w1 && v != -1 && !valid) && lane == 0) atomicOr(&g_dg_error, 0x2);
+      const unsigned same = __match_any_sync(0xffffffffu, valid ? v : -1);
+      if (valid && (same & lt) == 0u) row[v] += __popc(same);
+      __syncwarp();
     }
   }
-  auto id_at = [&](int i) -> int {
-    if constexpr (kStaged) return ids_s[i];
-    else return __ldg(&ids[i]);
-  };
   __syncthreads();
-  // 1. this CTA's slice: counts (lanes holding the same id add once per warp),
-  //    unrouted and out-of-range slots
-  const int slice = (n + kRouteCluster - 1) / kRouteCluster;
-  const int s0 = min(n, crank * slice), s1 = min(n, s0 + slice);
-  for (int base = s0; base < s1; base += blockDim.x) {
-    const int i = base + tid;
-    const int v = i < s1 ? id_at(i) : -1;
-    if (i < s1 && (v < 0 || v >= G)) row_of[i] = -1;
-    if (__any_sync(0xffffffffu, i < s1 && !(v >= -1 && v < G)) && lane == 0) atomicOr(&g_dg_error, 0x2);
-    const unsigned same = __match_any_sync(0xffffffffu, v);
-    if (v >= 0 && v < G && lane == __ffs(same) - 1) atomicAdd(&cnt[v], __popc(same));
+  // 2. prefixes over the warps, slice counts, then the cluster's sums
+  for (int e = tid; e < G; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int t = wtab[w * G + e];
+      wtab[w * G + e] = run;
+      run += t;
+    }
+    ccnt[e] = run;
   }
   cluster_sync();
-  // 2. the histogram: the sum of the cluster's slice counts
-  for (int g = tid; g < G; g += blockDim.x) {
-    const uint32_t a = smem_u32(&cnt[g]);
-    int t = 0;
+  for (int e = tid; e < G; e += blockDim.x) {
+    const uint32_t a = smem_u32(&ccnt[e]);
+    int t = 0, b = 0;
 #pragma unroll
-    for (int c = 0; c < kRouteCluster; ++c) t += static_cast<int>(ld_shared_cluster_u32(mapa_shared(a, c)));
-    tot[g] = t;
-  }
-  cluster_sync();  // every CTA has read every slice: from here none reads a peer
-  if (tid == 0) {
-    int off = 0, all = 0;
-    for (int g = 0; g < G; ++g) {
-      const int padded = (tot[g] + 127) & ~127;
-      if (g < e) off += padded;
-      all += padded;
+    for (int r = 0; r < kRouteCluster; ++r) {
+      const int x = static_cast<int>(ld_shared_cluster_u32(mapa_shared(a, r)));
+      t += x;
+      if (r < c) b += x;
     }
-    seg_off = off;
-    total_rows = all;
-    chunk_off[0] = 0;
+    tot[e] = t;
+    below[e] = b;
   }
-  __syncthreads();
-  if (e >= G) return;  // a CTA that only completes the last cluster
-  // 3. stable compaction of the slots routed to expert e
-  int par = 0;
-  for (int base = 0; base < n; base += 16 * kMoeThreads, par ^= 1) {
-    const int i0 = base + 16 * tid;
-    unsigned flags = 0;
-    if (kStaged && i0 + 15 < n) {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int4 v4 = reinterpret_cast<const int4*>(ids_s + i0)[q];  // i0 is a multiple of 16: aligned
-        flags |= (static_cast<unsigned>(v4.x == e) | (static_cast<unsigned>(v4.y == e) << 1) |
-                  (static_cast<unsigned>(v4.z == e) << 2) | (static_cast<unsigned>(v4.w == e) << 3))
-                 << (4 * q);
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int i = i0 + j;
-        flags |= static_cast<unsigned>(i < n && id_at(i) == e) << j;
-      }
-    }
-    const int c = __popc(flags);
-    int incl = c;
+  cluster_sync();  // every CTA has read every slice count: from here none reads a peer
+  // 3. segment offsets: exclusive scan of the padded totals (G <= blockDim)
+  {
+    const int v = tid < G ? (tot[tid] + 127) & ~127 : 0;
+    int incl = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int u = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += u;
     }
-    if (lane == 31) warp_tot[par][warp] = incl;
+    if (lane == 31) warp_sum[warp] = incl;
     __syncthreads();
     if (warp == 0) {
-      const int v = lane < nw ? warp_tot[par][lane] : 0;
-      int x = v;
+      const int x = warp_sum[lane];
+      int y = x;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int u = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += u;
+        const int u = __shfl_up_sync(0xffffffffu, y, o);
+        if (lane >= o) y += u;
       }
-      if (lane < nw) warp_tot[par][lane] = x - v;  // exclusive prefix of the warps
-      if (lane == 31) chunk_off[par ^ 1] = chunk_off[par] + x;
+      warp_sum[lane] = y - x;
+      if (lane == 31) total_rows_s = y;
     }
     __syncthreads();
-    int pos = seg_off + chunk_off[par] + warp_tot[par][warp] + incl - c;
-    while (flags != 0u) {
-      const int i = i0 + __ffs(flags) - 1;
-      flags &= flags - 1u;
-      m_indices[pos] = e;
-      src_of[pos] = i / topk;
-      row_of[i] = pos;
-      ++pos;
+    if (tid < G) seg[tid] = warp_sum[warp] + incl - v;
+    __syncthreads();
+  }
+  for (int i = tid; i < 32 * G; i += blockDim.x) {
+    const int e = i % G;
+    wtab[i] += seg[e] + below[e];
+  }
+  __syncthreads();
+  // 4. rows of the routed slots, in slot order
+  for (int base = w0; base < w1; base += 32 * kRouteSteps) {
+    int vs[kRouteSteps];
+#pragma unroll
+    for (int j = 0; j < kRouteSteps; ++j) {
+      const int i = base + 32 * j + lane;
+      vs[j] = i < w1 ? __ldg(&ids[i]) : -1;
+    }
+#pragma unroll
+    for (int j = 0; j < kRouteSteps; ++j) {
+      const int i = base + 32 * j + lane;
+      const int v = vs[j];
+      const bool valid = v >= 0 && v < G;
+      const unsigned same = __match_any_sync(0xffffffffu, valid ? v : -1);
+      const int pos = valid ? row[v] + __popc(same & lt) : 0;
+      __syncwarp();
+      if (valid && (same & lt) == 0u) row[v] += __popc(same);
+      __syncwarp();
+      if (valid) {
+        m_indices[pos] = v;
+        src_of[pos] = i / topk;
+        row_of[i] = pos;
+      }
     }
   }
-  // padding rows of this segment (scale words 0); CTA 0 also marks the tail past the last segment
-  const int c = tot[e];
-  const int pad0 = seg_off + c, pad1 = seg_off + ((c + 127) & ~127);
-  for (int r = pad0 + tid; r < pad1; r += blockDim.x) {
-    m_indices[r] = -1;
-    src_of[r] = -1;
-  }
-  for (int u = tid; u < (pad1 - pad0) * kp; u += blockDim.x)
-    sfa_perm[static_cast<size_t>(u / (pad1 - pad0)) * M_cap + pad0 + u % (pad1 - pad0)] = 0u;
-  if (e == 0) {
-    for (int r = total_rows + tid; r < M_cap; r += blockDim.x) {
+  // 5. padding rows of the segments of experts c, c + C, ..., and a share of the tail
+  for (int e = c; e < G; e += kRouteCluster) {
+    const int pad0 = seg[e] + tot[e], pad1 = seg[e] + ((tot[e] + 127) & ~127);
+    for (int r = pad0 + tid; r < pad1; r += blockDim.x) {
       m_indices[r] = -1;
       src_of[r] = -1;
+      for (int k = 0; k < kp; ++k) sfa_perm[static_cast<size_t>(k) * M_cap + r] = 0u;
     }
-    const int tail = M_cap - total_rows;
-    for (long long u = tid; u < static_cast<long long>(tail) * kp; u += blockDim.x)
-      sfa_perm[static_cast<size_t>(u / tail) * M_cap + total_rows + u % tail] = 0u;
+  }
+  for (int r = total_rows_s + c * blockDim.x + tid; r < M_cap; r += kRouteCluster * blockDim.x) {
+    m_indices[r] = -1;
+    src_of[r] = -1;
+    for (int k = 0; k < kp; ++k) sfa_perm[static_cast<size_t>(k) * M_cap + r] = 0u;
   }
 }
 
 // a_perm[row_of[t][s]] = q[t] (K bytes) and sfa_perm[kp][row_of[t][s]] =
 // sfa[kp][t] for every routed slot s of token t: tokens in source order, so
-// each token's row is read once however many slots it has.  Padding and tail
+// each token's row is read once however many slots it has.  Each thread takes
+// kGatherU 16-byte units per pass (stride apart), loading all of them before
+// storing any, so several loads are in flight per thread.  Padding and tail
 // rows keep whatever codes they held (their scale words are zeroed by
 // moe_route_kernel).
+constexpr int kGatherU = 4;
 __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restrict__ q, const uint32_t* __restrict__ sfa,
                                                         int T, int K, int kp, int topk,
                                                         const int32_t* __restrict__ row_of, int M_cap,
@@ -201,22 +213,39 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
   const int chunks = K / 16;
   const int t4 = (T + 3) & ~3;
   const long long total = static_cast<long long>(T) * chunks;
-  for (long long u = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u < total;
-       u += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(u / chunks);
-    const int ch = static_cast<int>(u - static_cast<long long>(t) * chunks);
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + static_cast<size_t>(t) * K) + ch);
-    const uint32_t w = ch < kp ? __ldg(&sfa[static_cast<size_t>(ch) * t4 + t]) : 0u;
-    for (int s = 0; s < topk; ++s) {
-      const int r = __ldg(&row_of[static_cast<size_t>(t) * topk + s]);
-      if (r < 0) continue;
-      reinterpret_cast<uint4*>(a_perm + static_cast<size_t>(r) * K)[ch] = v;
-      if (ch < kp) sfa_perm[static_cast<size_t>(ch) * M_cap + r] = w;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long u0 = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; u0 < total;
+       u0 += kGatherU * stride) {
+    int t[kGatherU], ch[kGatherU];
+    uint4 v[kGatherU];
+    uint32_t w[kGatherU];
+#pragma unroll
+    for (int j = 0; j < kGatherU; ++j) {
+      const long long u = u0 + j * stride;
+      t[j] = u < total ? static_cast<int>(u / chunks) : -1;
+      ch[j] = u < total ? static_cast<int>(u - static_cast<long long>(t[j]) * chunks) : 0;
+      v[j] = t[j] >= 0 ? __ldg(reinterpret_cast<const uint4*>(q + static_cast<size_t>(t[j]) * K) + ch[j])
+                       : make_uint4(0, 0, 0, 0);
+      w[j] = t[j] >= 0 && ch[j] < kp ? __ldg(&sfa[static_cast<size_t>(ch[j]) * t4 + t[j]]) : 0u;
+    }
+#pragma unroll
+    for (int j = 0; j < kGatherU; ++j) {
+      if (t[j] < 0) continue;
+      for (int s = 0; s < topk; ++s) {
+        const int r = __ldg(&row_of[static_cast<size_t>(t[j]) * topk + s]);
+        if (r < 0) continue;
+        reinterpret_cast<uint4*>(a_perm + static_cast<size_t>(r) * K)[ch[j]] = v[j];
+        if (ch[j] < kp) sfa_perm[static_cast<size_t>(ch[j]) * M_cap + r] = w[j];
+      }
     }
   }
 }
 
-// One thread per (token, 8 output columns).
+// One thread per (token, 8 output columns).  The slots of the token are
+// taken kSlots at a time: first their row indices and weights, then all of
+// their 16-byte row loads, then the FP32 sums in slot order, so a thread has
+// up to kSlots row loads in flight at once.
+template <int kSlots>
 __global__ void __launch_bounds__(256) moe_combine_kernel(const __nv_bfloat16* __restrict__ d, const int32_t* __restrict__ row_of,
                                                          const float* __restrict__ w, int T, int topk, int N,
                                                          __nv_bfloat16* __restrict__ out) {
@@ -229,16 +258,30 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const __nv_bfloat16* _
     const int t = static_cast<int>(u / chunks);
     const int ch = static_cast<int>(u - static_cast<long long>(t) * chunks);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    for (int s = 0; s < topk; ++s) {
-      const int r = __ldg(&row_of[t * topk + s]);
-      if (r < 0) continue;
-      const float ws = w ? __ldg(&w[t * topk + s]) : 1.0f;
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(d + static_cast<size_t>(r) * N) + ch);
-      const uint32_t u32[4] = {v.x, v.y, v.z, v.w};
+    for (int s0 = 0; s0 < topk; s0 += kSlots) {
+      int r[kSlots];
+      float ws[kSlots];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc[2 * i] = fmaf(ws, __uint_as_float(u32[i] << 16), acc[2 * i]);
-        acc[2 * i + 1] = fmaf(ws, __uint_as_float(u32[i] & 0xFFFF0000u), acc[2 * i + 1]);
+      for (int q = 0; q < kSlots; ++q) {
+        const bool ok = s0 + q < topk;
+        const size_t at = static_cast<size_t>(t) * topk + s0 + q;
+        r[q] = ok ? __ldg(&row_of[at]) : -1;
+        ws[q] = ok && w ? __ldg(&w[at]) : 1.0f;
+      }
+      uint4 v[kSlots];
+#pragma unroll
+      for (int q = 0; q < kSlots; ++q)
+        v[q] = r[q] >= 0 ? __ldg(reinterpret_cast<const uint4*>(d + static_cast<size_t>(r[q]) * N) + ch)
+                         : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int q = 0; q < kSlots; ++q) {
+        if (r[q] < 0) continue;
+        const uint32_t u32[4] = {v[q].x, v[q].y, v[q].z, v[q].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          acc[2 * i] = fmaf(ws[q], __uint_as_float(u32[i] << 16), acc[2 * i]);
+          acc[2 * i + 1] = fmaf(ws[q], __uint_as_float(u32[i] & 0xFFFF0000u), acc[2 * i + 1]);
+        }
       }
     }
     uint32_t o[4];

@@ -114,6 +114,30 @@ def test_permute_flags_bad_ids():
     assert out["row_of"].cpu().numpy().tolist() == [[0, -1], [128, -1]]
 
 
+@pytest.mark.parametrize("T,topk,N,weighted", [(1, 1, 16, True), (333, 2, 272, True), (257, 3, 4096, False),
+                                                (100, 6, 512, True), (64, 8, 128, True), (50, 9, 96, True),
+                                                (20, 12, 48, False)])
+def test_combine_matches_oracle(T, topk, N, weighted):
+    """The weighted combine on its own, over every slot-pass width (top-k 1, 2,
+    3 -> 4, 6 -> 8, 8, and 9 / 12, which take two passes of 8), with unrouted
+    slots, a token with no routed slot, and rows of the permuted output that
+    no slot reads."""
+    rng = np.random.default_rng(T * 31 + topk)
+    R = T * topk + 37
+    d = torch.from_numpy(synth.normal(T + topk, R * N).reshape(R, N)).to(torch.bfloat16).cuda()
+    row_of = rng.permutation(R)[: T * topk].reshape(T, topk).astype(np.int32)
+    row_of[rng.random((T, topk)) < 0.15] = -1
+    row_of[T // 2] = -1
+    gate = rng.random((T, topk)).astype(np.float32) if weighted else None
+    out = torch.full((T, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    dg.moe_unpermute_combine(d, torch.from_numpy(row_of).cuda(), torch.from_numpy(gate).cuda() if weighted else None,
+                             out=out)
+    torch.cuda.synchronize()
+    ref = oracle.fp8_gemm.moe_unpermute_combine(bits(d), row_of, gate)
+    check_close(bits(out), ref, "combine")
+    assert (bits(out)[T // 2] == 0).all()
+
+
 def test_moe_chain_matches_oracle():
     T, topk, G, K, N = 700, 2, 5, 1024, 384
     ids = _routing(T, topk, G, seed=3, drop=0.05)
