@@ -801,6 +801,21 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
         acc_use = local_tile / L::kNumAcc;
       }
       ++local_tile;
+      // FP32 output plus C (dense only): the C values of the warp's chunks are
+      // loaded one chunk ahead, the first before the accumulator is ready, so
+      // their latency overlaps the MMAs and the previous chunk's stores.
+      float4 cbuf[2][8];
+      const bool c_rows = OUT_F32 && MODE == MODE_DENSE && p.c != nullptr &&
+                          tl.row0 + 128 * static_cast<int>(rank) + 32 * q + lane < p.rows;
+      auto load_c = [&](int col0, float4 (&cv)[8]) {
+        const float4* cp = reinterpret_cast<const float4*>(
+            p.c + static_cast<size_t>(tl.row0 + 128 * static_cast<int>(rank) + 32 * q + lane) * p.N + col0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cv[i] = col0 + 4 * i < p.N ? __ldg(cp + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+      };
+      if constexpr (OUT_F32) {
+        if (c_rows && nmine > 0 && tl.n_blk * BN + 32 * half < p.N) load_c(tl.n_blk * BN + 32 * half, cbuf[0]);
+      }
       bool ok = wait_phase<false>(&tmem_full[acc], acc_use & 1, abort_flag, p.wait_limit_ns);
       if (split && ok) ok = wait_phase<false>(&tmem_full[1], uses1++ & 1, abort_flag, p.wait_limit_ns);
       ok = __all_sync(0xffffffffu, ok);
@@ -829,19 +844,17 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(32 * q) << 16) + acc * L::kAccStride;
 
       // Converts and stores one 32-column chunk held in rr (lane = row).
-      auto store_chunk = [&](uint32_t (&rr)[32], int col0) {
+      auto store_chunk = [&](uint32_t (&rr)[32], int col0, const float4 (&cv)[8]) {
         if constexpr (OUT_F32) {
-          // FP32 output, optionally plus C: two 16-column halves of 64 B per row
-          if (p.c != nullptr && valid) {
-            const float4* cp = reinterpret_cast<const float4*>(p.c + row_g * p.N + col0);
+          // FP32 output, optionally plus C (prefetched into cv): two 16-column halves of 64 B per row
+          if (c_rows) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               if (col0 + 4 * i < p.N) {
-                const float4 cv = __ldg(cp + i);
-                rr[4 * i] = __float_as_uint(__uint_as_float(rr[4 * i]) + cv.x);
-                rr[4 * i + 1] = __float_as_uint(__uint_as_float(rr[4 * i + 1]) + cv.y);
-                rr[4 * i + 2] = __float_as_uint(__uint_as_float(rr[4 * i + 2]) + cv.z);
-                rr[4 * i + 3] = __float_as_uint(__uint_as_float(rr[4 * i + 3]) + cv.w);
+                rr[4 * i] = __float_as_uint(__uint_as_float(rr[4 * i]) + cv[i].x);
+                rr[4 * i + 1] = __float_as_uint(__uint_as_float(rr[4 * i + 1]) + cv[i].y);
+                rr[4 * i + 2] = __float_as_uint(__uint_as_float(rr[4 * i + 2]) + cv[i].z);
+                rr[4 * i + 3] = __float_as_uint(__uint_as_float(rr[4 * i + 3]) + cv[i].w);
               }
             }
           }
@@ -978,7 +991,12 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
           const int c = half + 2 * i;
           const int col0 = n0 + 32 * c;
           if (i >= nmine || col0 >= p.N) break;
-          if (i + 1 < nmine && col0 + 64 < p.N) tmem_ld_32x32b_x32(t_row + 32 * (c + 2), r[(i + 1) & 1]);
+          if (i + 1 < nmine && col0 + 64 < p.N) {
+            tmem_ld_32x32b_x32(t_row + 32 * (c + 2), r[(i + 1) & 1]);
+            if constexpr (OUT_F32) {
+              if (c_rows) load_c(col0 + 64, cbuf[(i + 1) & 1]);
+            }
+          }
           if (split) {
             // a split tile: add the second pipeline's accumulator, 16 columns at a time
 #pragma unroll
@@ -992,7 +1010,7 @@ __global__ void __launch_bounds__(kThreadsFor<PIPES>, 1)
                     __float_as_uint(__uint_as_float(r[i & 1][16 * hh + j]) + __uint_as_float(h[j]));
             }
           }
-          store_chunk(r[i & 1], col0);
+          store_chunk(r[i & 1], col0, cbuf[i & 1]);
           tmem_wait_ld();
         }
       }
