@@ -898,14 +898,14 @@ int dg_moe_unpermute_combine(const void* d_perm, const int32_t* row_of, const fl
   DeviceInfo di;
   int r = device_info(&di);
   if (r) return r;
-  // slots per pass: one at a time up to top-2 (measured fastest there), else 4 or 8 (passes of 8 beyond)
-  const int slots = topk <= 2 ? 1 : topk <= 4 ? 4 : 8;
+  // slots per pass: one at a time up to top-4, else 8 (passes of 8 beyond top-8); measured
+  // fastest on top-2 and top-4 (N = 4096) and on top-8 (N = 7168) respectively
+  const int slots = topk <= 4 ? 1 : 8;
   const long long blocks = std::max<long long>(1, std::min<long long>((work + 255) / 256, 16LL * di.sms));
   auto st = static_cast<cudaStream_t>(stream);
   auto dp = static_cast<const __nv_bfloat16*>(d_perm);
   auto op = static_cast<__nv_bfloat16*>(out);
   if (slots == 1) DG_CUDA_TRY(launch_plain(moe_combine_kernel<1>, blocks, 256, st, dp, row_of, weights, T, topk, N, op));
-  else if (slots == 4) DG_CUDA_TRY(launch_plain(moe_combine_kernel<4>, blocks, 256, st, dp, row_of, weights, T, topk, N, op));
   else DG_CUDA_TRY(launch_plain(moe_combine_kernel<8>, blocks, 256, st, dp, row_of, weights, T, topk, N, op));
   return DG_OK;
 }

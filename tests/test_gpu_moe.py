@@ -118,10 +118,10 @@ def test_permute_flags_bad_ids():
                                                 (100, 6, 512, True), (64, 8, 128, True), (50, 9, 96, True),
                                                 (20, 12, 48, False)])
 def test_combine_matches_oracle(T, topk, N, weighted):
-    """The weighted combine on its own, over every slot-pass width (top-k 1, 2,
-    3 -> 4, 6 -> 8, 8, and 9 / 12, which take two passes of 8), with unrouted
-    slots, a token with no routed slot, and rows of the permuted output that
-    no slot reads."""
+    """The weighted combine on its own, over both slot-pass widths (one slot at
+    a time for top-k 1, 2, 3; eight for 6 and 8, and two passes of eight for 9
+    and 12), with unrouted slots, a token with no routed slot, and rows of the
+    permuted output that no slot reads."""
     rng = np.random.default_rng(T * 31 + topk)
     R = T * topk + 37
     d = torch.from_numpy(synth.normal(T + topk, R * N).reshape(R, N)).to(torch.bfloat16).cuda()
