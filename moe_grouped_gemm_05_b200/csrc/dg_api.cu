@@ -883,8 +883,9 @@ int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, co
   const long long blocks =
       std::max<long long>(1, std::min<long long>((work + 256 * kGatherU - 1) / (256 * kGatherU), 8LL * di.sms));
   DG_CUDA_TRY(launch_plain(moe_gather_kernel, blocks, 256, st, static_cast<const uint8_t*>(q),
-                           reinterpret_cast<const uint32_t*>(sfa), T, K, kp, topk, static_cast<const int32_t*>(row_of),
-                           M_cap, static_cast<uint8_t*>(a_perm), reinterpret_cast<uint32_t*>(sfa_perm)));
+                           reinterpret_cast<const uint32_t*>(sfa), T, K, kp, topk, topk_ids,
+                           static_cast<const int32_t*>(row_of), M_cap, static_cast<uint8_t*>(a_perm),
+                           reinterpret_cast<uint32_t*>(sfa_perm), m_indices, src_of));
   return DG_OK;
 }
 

@@ -9,11 +9,12 @@
 //                    CTAs add their counts through distributed shared memory
 //                    -> each expert's segment offset (segments in expert
 //                    order, each padded to 128 rows), so the layout is
-//                    deterministic.  Writes m_indices, src_of, row_of, and
-//                    zero scale words for padding rows.
+//                    deterministic.  Writes row_of, and m_indices, src_of
+//                    and zero scale words for padding rows.
 // moe_gather_kernel  full grid, tokens in source order: copies each token's
 //                    FP8 codes and packed scale words to the rows of its
-//                    routed slots (one read of each token row).
+//                    routed slots (one read of each token row), and writes
+//                    those rows' expert and source token.
 // moe_combine_kernel out[t] = bf16(sum_s w[t,s] * D[row_of[t,s]]), FP32 sums.
 #pragma once
 #include <cuda_bf16.h>
@@ -36,12 +37,28 @@ constexpr int kRouteSteps = 8;
 // earlier CTAs' counts and the segment offsets (G words each).
 __host__ __device__ constexpr int route_smem_bytes(int G) { return (32 * G + 4 * G) * 4; }
 
+// Lanes of the warp whose key equals this lane's, for keys in [0, 2^nbits).
+// Keys of up to 6 bits: match.any; wider: the AND over the key's bits of the
+// ballot of the lanes agreeing on that bit (nbits ballots).  In the routing
+// kernel's first pass the ballots measured faster with 256 experts (15.0 ->
+// 11.8 us) and slower with 8 (2.4 -> 3.7 us).
+__device__ __forceinline__ unsigned warp_same_key(int key, int nbits) {
+  if (nbits <= 6) return __match_any_sync(0xffffffffu, key);
+  unsigned m = 0xffffffffu;
+  for (int b = 0; b < nbits; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned bal = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? bal : ~bal;
+  }
+  return m;
+}
+
 // A stable counting sort of the n routed slots by expert, on one cluster of
 // kRouteCluster CTAs of 32 warps.  CTA c owns slots [c*slice, (c+1)*slice),
 // and warp w of it a run of that range in slot order (whole 32-slot steps).
-// 1. every warp counts the slots of its run per expert (match_any: lanes
-//    with the same expert add once, by their first lane), into its row of
-//    the table; unrouted and invalid slots get row_of = -1;
+// 1. every warp counts the slots of its run per expert (lanes with the same
+//    expert add once, by their first lane), into its row of the table;
+//    unrouted and invalid slots get row_of = -1;
 // 2. the CTA turns the table into exclusive prefixes over its warps and its
 //    slice counts; the cluster adds every CTA's slice counts through
 //    distributed shared memory, giving the expert totals and, per expert,
@@ -51,9 +68,12 @@ __host__ __device__ constexpr int route_smem_bytes(int G) { return (32 * G + 4 *
 //    of expert e;
 // 4. every warp walks its run again in slot order: a slot's row is its
 //    warp's entry plus its rank among the lanes of the step with the same
-//    expert, and the first such lane advances the entry;
-// 5. the padding rows of the segments (experts split over the CTAs) and the
-//    rows past the last segment get index -1 and zero scale words.
+//    expert, and the first such lane advances the entry; only row_of is
+//    written here (coalesced): moe_gather_kernel, on the whole GPU, writes
+//    m_indices and src_of of the routed rows from it;
+// 5. the padding rows of the segments (one warp per expert, experts split
+//    over the CTAs) and the rows past the last segment get index -1 and zero
+//    scale words.
 __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int topk,
                                                                 int G, int M_cap, int kp, int32_t* __restrict__ m_indices,
                                                                 int32_t* __restrict__ row_of,
@@ -76,6 +96,7 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
   const int per_warp = ((s1 - s0 + 32 * 32 - 1) / (32 * 32)) * 32;  // whole 32-slot steps
   const int w0 = min(s1, s0 + warp * per_warp), w1 = min(s1, w0 + per_warp);
   const unsigned lt = (1u << lane) - 1u;
+  const int nbits = 32 - __clz(G);  // keys 0..G (G: unrouted or invalid)
   for (int i = tid; i < 32 * G; i += blockDim.x) wtab[i] = 0;
   __syncthreads();
   // 1. per-warp counts (the ids of kRouteSteps steps are loaded at once)
@@ -94,7 +115,7 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
       const bool valid = v >= 0 && v < G;
       if (i < w1 && !valid) row_of[i] = -1;
       if (__any_sync(0xffffffffu, i < w1 && v != -1 && !valid) && lane == 0) atomicOr(&g_dg_error, 0x2);
-      const unsigned same = __match_any_sync(0xffffffffu, valid ? v : -1);
+      const unsigned same = warp_same_key(valid ? v : G, nbits);
       if (valid && (same & lt) == 0u) row[v] += __popc(same);
       __syncwarp();
     }
@@ -168,22 +189,19 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
       const int i = base + 32 * j + lane;
       const int v = vs[j];
       const bool valid = v >= 0 && v < G;
-      const unsigned same = __match_any_sync(0xffffffffu, valid ? v : -1);
+      const unsigned same = warp_same_key(valid ? v : G, nbits);
       const int pos = valid ? row[v] + __popc(same & lt) : 0;
       __syncwarp();
       if (valid && (same & lt) == 0u) row[v] += __popc(same);
       __syncwarp();
-      if (valid) {
-        m_indices[pos] = v;
-        src_of[pos] = i / topk;
-        row_of[i] = pos;
-      }
+      if (valid) row_of[i] = pos;
     }
   }
-  // 5. padding rows of the segments of experts c, c + C, ..., and a share of the tail
-  for (int e = c; e < G; e += kRouteCluster) {
+  // 5. padding rows of the segments of experts c, c + C, ... (one warp per
+  //    expert), and a share of the tail
+  for (int e = c + kRouteCluster * warp; e < G; e += kRouteCluster * 32) {
     const int pad0 = seg[e] + tot[e], pad1 = seg[e] + ((tot[e] + 127) & ~127);
-    for (int r = pad0 + tid; r < pad1; r += blockDim.x) {
+    for (int r = pad0 + lane; r < pad1; r += 32) {
       m_indices[r] = -1;
       src_of[r] = -1;
       for (int k = 0; k < kp; ++k) sfa_perm[static_cast<size_t>(k) * M_cap + r] = 0u;
@@ -196,8 +214,9 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
   }
 }
 
-// a_perm[row_of[t][s]] = q[t] (K bytes) and sfa_perm[kp][row_of[t][s]] =
-// sfa[kp][t] for every routed slot s of token t: tokens in source order, so
+// a_perm[row_of[t][s]] = q[t] (K bytes), sfa_perm[kp][row_of[t][s]] =
+// sfa[kp][t], m_indices[row_of[t][s]] = ids[t][s] and src_of[row_of[t][s]] =
+// t for every routed slot s of token t: tokens in source order, so
 // each token's row is read once however many slots it has.  Each thread takes
 // kGatherU 16-byte units per pass (stride apart), loading all of them before
 // storing any, so several loads are in flight per thread.  Padding and tail
@@ -206,8 +225,10 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
 constexpr int kGatherU = 4;
 __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restrict__ q, const uint32_t* __restrict__ sfa,
                                                         int T, int K, int kp, int topk,
+                                                        const int32_t* __restrict__ ids,
                                                         const int32_t* __restrict__ row_of, int M_cap,
-                                                        uint8_t* __restrict__ a_perm, uint32_t* __restrict__ sfa_perm) {
+                                                        uint8_t* __restrict__ a_perm, uint32_t* __restrict__ sfa_perm,
+                                                        int32_t* __restrict__ m_indices, int32_t* __restrict__ src_of) {
   grid_dep_wait();
   grid_dep_launch();
   const int chunks = K / 16;
@@ -236,6 +257,10 @@ __global__ void __launch_bounds__(256) moe_gather_kernel(const uint8_t* __restri
         if (r < 0) continue;
         reinterpret_cast<uint4*>(a_perm + static_cast<size_t>(r) * K)[ch[j]] = v[j];
         if (ch[j] < kp) sfa_perm[static_cast<size_t>(ch[j]) * M_cap + r] = w[j];
+        if (ch[j] == 0) {
+          m_indices[r] = __ldg(&ids[static_cast<size_t>(t[j]) * topk + s]);
+          src_of[r] = t[j];
+        }
       }
     }
   }
