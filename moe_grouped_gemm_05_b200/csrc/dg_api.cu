@@ -876,7 +876,7 @@ int dg_moe_permute(const int32_t* topk_ids, int T, int topk, int num_experts, co
   }
   DG_CUDA_TRY(launch_plain_smem(moe_route_kernel, kRouteCluster, kMoeThreads,
                                 static_cast<size_t>(route_smem_bytes(num_experts)), st, kRouteCluster, topk_ids,
-                                static_cast<int>(n), topk, num_experts, M_cap, kp, m_indices, row_of, src_of,
+                                static_cast<int>(n), num_experts, M_cap, kp, m_indices, row_of, src_of,
                                 reinterpret_cast<uint32_t*>(sfa_perm)));
   const long long work = static_cast<long long>(T) * (K / 16);
   if (work == 0) return DG_OK;

@@ -74,7 +74,7 @@ __device__ __forceinline__ unsigned warp_same_key(int key, int nbits) {
 // 5. the padding rows of the segments (one warp per expert, experts split
 //    over the CTAs) and the rows past the last segment get index -1 and zero
 //    scale words.
-__global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n, int topk,
+__global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* __restrict__ ids, int n,
                                                                 int G, int M_cap, int kp, int32_t* __restrict__ m_indices,
                                                                 int32_t* __restrict__ row_of,
                                                                 int32_t* __restrict__ src_of,

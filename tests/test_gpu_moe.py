@@ -54,6 +54,35 @@ def test_permute_bit_exact(T, topk, G, K):
     assert (sf_out[:, gm < 0] == 0).all()
 
 
+@pytest.mark.parametrize("T,topk,G,K,zipf", [(20000, 8, 1024, 128, False), (40000, 2, 8, 128, True),
+                                               (3000, 4, 63, 256, False), (3000, 4, 64, 256, False)])
+def test_permute_many_slots_and_expert_counts(T, topk, G, K, zipf):
+    """Routing beyond 65536 slots (each warp of the routing cluster then loads
+    its ids in several batches), the largest expert count (1024: the 128 KB
+    per-warp count table), and 63 / 64 experts, on either side of the switch
+    from match.any to per-bit ballots (6- and 7-bit expert keys)."""
+    if zipf:
+        ids, _ = synth.topk_routing(T + G, T, topk, G)
+    else:
+        ids = _routing(T, topk, G, seed=T + G, drop=0.05)
+    x = torch.from_numpy(synth.normal(T + 1, T * K).reshape(T, K)).to(torch.bfloat16).cuda()
+    q, sfa = dg.quantize_fp8_1x128(x)
+    out = dg.moe_permute(torch.from_numpy(ids).cuda(), G, q, sfa)
+    torch.cuda.synchronize()
+    assert dg.get_device_error() == 0
+    m, row_of, src, Mt, bad = oracle.fp8_gemm.moe_permute(ids, G)
+    gm, gs = out["m_indices"].cpu().numpy(), out["src_of"].cpu().numpy()
+    assert np.array_equal(gm[:Mt], m) and (gm[Mt:] == -1).all()
+    assert np.array_equal(gs[:Mt], src) and (gs[Mt:] == -1).all()
+    assert np.array_equal(out["row_of"].cpu().numpy(), row_of)
+    valid = np.nonzero(m >= 0)[0]
+    an = out["a"].view(torch.uint8).cpu().numpy()
+    assert np.array_equal(an[valid], q.view(torch.uint8).cpu().numpy()[src[valid]])
+    sf_out = out["sfa"].cpu().numpy()
+    assert np.array_equal(sf_out[:, valid], sfa.cpu().numpy()[:, src[valid]])
+    assert (sf_out[:, gm < 0] == 0).all()
+
+
 def test_permute_into_prefilled_buffers_over_many_chunks():
     """15000 routed slots (several 4096-slot compaction chunks and a ragged
     last one) with Zipf-weighted top-3 routing, into output buffers filled with
