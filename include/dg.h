@@ -207,6 +207,8 @@ int dg_quantize_fp8_1x128(const void* x, int x_dtype, void* q, int32_t* sf, int 
  * of 128; inside a segment slots keep their (token, slot) order, so the result is
  * deterministic.  Rows past the last segment are -1.  a_perm / sfa_perm / m_indices
  * feed dg_m_grouped_fp8_gemm_nt_contiguous with M_total = M_cap directly.
+ * The codes of padding and tail rows of a_perm are not written (their scale words
+ * are written as 0, and the grouped GEMM never stores those rows).
  * Ids outside [-1, num_experts) set DG_DEVERR_BAD_EXPERT and are not routed.
  * num_experts <= 1024; M_cap >= dg_moe_permute_capacity(...) and a multiple of 128.
  * With T = 0, topk_ids, q, sfa and row_of may be NULL: every row becomes padding.
