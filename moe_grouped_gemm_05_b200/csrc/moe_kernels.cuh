@@ -99,9 +99,13 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
   const int nbits = 32 - __clz(G);  // keys 0..G (G: unrouted or invalid)
   for (int i = tid; i < 32 * G; i += blockDim.x) wtab[i] = 0;
   __syncthreads();
-  // 1. per-warp counts (the ids of kRouteSteps steps are loaded at once)
+  // 1. per-warp counts (the ids of kRouteSteps steps are loaded at once; the
+  //    first batch's ids and same-expert masks stay in registers for step 4)
   int* row = wtab + warp * G;
+  int vs0[kRouteSteps];
+  unsigned ms0[kRouteSteps];
   for (int base = w0; base < w1; base += 32 * kRouteSteps) {
+    const bool first = base == w0;
     int vs[kRouteSteps];
 #pragma unroll
     for (int j = 0; j < kRouteSteps; ++j) {
@@ -118,6 +122,10 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
       const unsigned same = warp_same_key(valid ? v : G, nbits);
       if (valid && (same & lt) == 0u) row[v] += __popc(same);
       __syncwarp();
+      if (first) {
+        vs0[j] = v;
+        ms0[j] = same;
+      }
     }
   }
   __syncthreads();
@@ -178,18 +186,19 @@ __global__ void __launch_bounds__(kMoeThreads) moe_route_kernel(const int32_t* _
   __syncthreads();
   // 4. rows of the routed slots, in slot order
   for (int base = w0; base < w1; base += 32 * kRouteSteps) {
+    const bool first = base == w0;
     int vs[kRouteSteps];
 #pragma unroll
     for (int j = 0; j < kRouteSteps; ++j) {
       const int i = base + 32 * j + lane;
-      vs[j] = i < w1 ? __ldg(&ids[i]) : -1;
+      vs[j] = first ? vs0[j] : (i < w1 ? __ldg(&ids[i]) : -1);
     }
 #pragma unroll
     for (int j = 0; j < kRouteSteps; ++j) {
       const int i = base + 32 * j + lane;
       const int v = vs[j];
       const bool valid = v >= 0 && v < G;
-      const unsigned same = warp_same_key(valid ? v : G, nbits);
+      const unsigned same = first ? ms0[j] : warp_same_key(valid ? v : G, nbits);
       const int pos = valid ? row[v] + __popc(same & lt) : 0;
       __syncwarp();
       if (valid && (same & lt) == 0u) row[v] += __popc(same);
