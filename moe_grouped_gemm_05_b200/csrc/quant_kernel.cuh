@@ -88,11 +88,11 @@ __global__ void __launch_bounds__(256) quantize_1x128_kernel(const T* __restrict
   const int kb_total = K >> 7;
   for (long long u = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); u < units;
        u += warps) {
-    // units run row-fastest inside a K span so consecutive warps write consecutive scale words
-    const int m = static_cast<int>(u % mn4);
-    const long long rest = u / mn4;
-    const int p = static_cast<int>(rest % kp);
-    const int b = static_cast<int>(rest / kp);
+    // units run span-fastest along a row, so consecutive warps read and write consecutive bytes
+    const int p = static_cast<int>(u % kp);
+    const long long rest = u / kp;
+    const int m = static_cast<int>(rest % mn4);
+    const int b = static_cast<int>(rest / mn4);
     uint32_t word = 0;
     if (m < M) {
       const int j = lane >> 3;               // K block within the span
